@@ -1,0 +1,324 @@
+// rocs_oracle.cpp -- plain fp64 CPU oracle for IKBO-LCB and IKBO-DCA.
+//
+// TEST INFRASTRUCTURE ONLY.  This oracle is used by the tests, by the smoke check
+// and by the CPU-baseline leg of the benchmark.  The CUDA product path never links,
+// loads or calls it; it shares no code, header, table or helper with that path.
+//
+// What it computes follows "ROCS: Request-Oriented Compute Sharing for Efficient
+// Large-Scale Recommendation" (arXiv:2607.27744), as read from the paper-archivist
+// reading notes of that paper:
+//   * LCB: the two-group ROCSified linear compression block, section 3.1.2, Eq. (5)
+//     and its explicit two-group form Eq. (6):
+//         [Y^R; Y^C] = [[W_RR, 0], [W_CR, W_CC]] . [X^R; X^C]
+//     evaluated per candidate with the request-to-candidate broadcast MATERIALISED
+//     (each candidate gets a fresh copy of its request's X^R) -- the plain
+//     definition; the in-kernel broadcast of section 4 only reorders this sum.
+//   * the request-output identity of section 3.1.5, Eq. (11): the request rows of
+//     every candidate's full output equal the request output computed once; the
+//     oracle checks this exactly on every candidate it evaluates.
+//   * DCA: the candidate-group cross attention of section 3.2, Eq. (13),
+//         A^C = Attn(Q^C, K, V) = softmax(scale . Q^C K^T) V,
+//     non-causal, each candidate's query tokens over its own request's keys, with
+//     the K/V broadcast MATERIALISED per candidate (section 4.3 describes the
+//     dense implementation that copies K/V to the candidate batch).
+//   * the chained block used by the chained workload: LCB -> bf16 -> linear query
+//     projection -> bf16 -> DCA (section 3.2, Eq. (12): queries generated from the
+//     LCB output; the projection is a plain linear map, no bias, no activation).
+//
+// Everything accumulates in double, in the index order written in the loops below.
+// Inputs are widened to double exactly from their stored fp32 / bf16 bits.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+namespace {
+
+enum { ORC_OK = 0, ORC_INVALID = 1, ORC_BAD_OFFSETS = 2, ORC_ISOLATION = 10 };
+
+// exact widening of a stored element (dtype 0: fp32, 1: bf16 bit pattern)
+inline double widen(const void* base, int dtype, int64_t idx) {
+  if (dtype == 0) return (double)static_cast<const float*>(base)[idx];
+  uint32_t u = (uint32_t)static_cast<const uint16_t*>(base)[idx] << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+// Round a double to the nearest bf16 value (ties to even), returned as a double.
+// bf16 = 8 significant bits, exponent range of binary32 (normal min 2^-126,
+// subnormal quantum 2^-133).  Uses frexp + nearbyint (default rounding mode is
+// round-half-even), i.e. a single rounding straight from double.
+inline double round_bf16(double x) {
+  if (!std::isfinite(x) || x == 0.0) return x;
+  int e;
+  double m = std::frexp(x, &e);  // x = m * 2^e, 0.5 <= |m| < 1
+  int q = e - 8;                 // quantum exponent for 8 significant bits
+  if (q < -133) q = -133;
+  double r = std::nearbyint(std::ldexp(x, -q));
+  double v = std::ldexp(r, q);
+  if (std::fabs(v) >= std::ldexp(1.0, 128)) v = std::copysign(std::numeric_limits<double>::infinity(), x);
+  return v;
+}
+
+// CSR check: off[0] == 0, non-decreasing, off[R] == total (total < 0: skip that test).
+bool csr_ok(const int32_t* off, int64_t R, int64_t total) {
+  if (R < 0 || off == nullptr) return false;
+  if (off[0] != 0) return false;
+  for (int64_t r = 0; r < R; ++r)
+    if (off[r + 1] < off[r]) return false;
+  return total < 0 || (int64_t)off[R] == total;
+}
+
+// candidate -> request map m, derived by a linear walk over the offsets (section 4.1)
+std::vector<int64_t> index_map(const int32_t* off, int64_t R) {
+  std::vector<int64_t> m((size_t)off[R]);
+  for (int64_t r = 0; r < R; ++r)
+    for (int64_t i = off[r]; i < off[r + 1]; ++i) m[(size_t)i] = r;
+  return m;
+}
+
+void set_threads(int nthreads) {
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+}
+
+// ---- LCB, one candidate: Eq. (6) with the broadcast materialised ------------------------
+// y_full [(o_r+o_c) x d] = W_full [(o_r+o_c) x (n_r+n_c)] . X_full [(n_r+n_c) x d]
+struct LcbDims {
+  int64_t n_r, n_c, d, o_r, o_c;
+};
+
+void lcb_full_weight(const LcbDims& D, int dtype, const void* w_rr, const void* w_cr, const void* w_cc,
+                     std::vector<double>& W) {
+  const int64_t ni = D.n_r + D.n_c, no = D.o_r + D.o_c;
+  W.assign((size_t)(no * ni), 0.0);
+  for (int64_t o = 0; o < D.o_r; ++o) {
+    for (int64_t j = 0; j < D.n_r; ++j) W[(size_t)(o * ni + j)] = widen(w_rr, dtype, o * D.n_r + j);
+    for (int64_t j = 0; j < D.n_c; ++j) W[(size_t)(o * ni + D.n_r + j)] = 0.0;  // the masked block M_RC = 0
+  }
+  for (int64_t o = 0; o < D.o_c; ++o) {
+    for (int64_t j = 0; j < D.n_r; ++j) W[(size_t)((D.o_r + o) * ni + j)] = widen(w_cr, dtype, o * D.n_r + j);
+    for (int64_t j = 0; j < D.n_c; ++j) W[(size_t)((D.o_r + o) * ni + D.n_r + j)] = widen(w_cc, dtype, o * D.n_c + j);
+  }
+}
+
+// Y^R_r = W_RR . X^R_r, j ascending
+void lcb_request(const LcbDims& D, int dtype, const void* x_req, const std::vector<double>& W, int64_t r,
+                 double* y /* [o_r x d] */) {
+  const int64_t ni = D.n_r + D.n_c;
+  for (int64_t o = 0; o < D.o_r; ++o)
+    for (int64_t c = 0; c < D.d; ++c) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < D.n_r; ++j) acc += W[(size_t)(o * ni + j)] * widen(x_req, dtype, (r * D.n_r + j) * D.d + c);
+      y[o * D.d + c] = acc;
+    }
+}
+
+// Full output of candidate i.  Returns false if the request rows differ from Y^R (Eq. 11).
+bool lcb_candidate(const LcbDims& D, int dtype, const void* x_req, const void* x_cand, const std::vector<double>& W,
+                   int64_t i, int64_t r, double* y_cand /* [o_c x d] */) {
+  const int64_t ni = D.n_r + D.n_c, no = D.o_r + D.o_c;
+  // the explicit broadcast: a fresh copy X_full = [X^R_r ; X^C_i]
+  std::vector<double> X((size_t)(ni * D.d));
+  for (int64_t j = 0; j < D.n_r; ++j)
+    for (int64_t c = 0; c < D.d; ++c) X[(size_t)(j * D.d + c)] = widen(x_req, dtype, (r * D.n_r + j) * D.d + c);
+  for (int64_t j = 0; j < D.n_c; ++j)
+    for (int64_t c = 0; c < D.d; ++c) X[(size_t)((D.n_r + j) * D.d + c)] = widen(x_cand, dtype, (i * D.n_c + j) * D.d + c);
+  std::vector<double> Y((size_t)(no * D.d));
+  for (int64_t o = 0; o < no; ++o)
+    for (int64_t c = 0; c < D.d; ++c) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < ni; ++j) acc += W[(size_t)(o * ni + j)] * X[(size_t)(j * D.d + c)];
+      Y[(size_t)(o * D.d + c)] = acc;
+    }
+  // Eq. (11): request rows of the full output == Y^R of the request, computed alone
+  std::vector<double> yr((size_t)(D.o_r * D.d));
+  lcb_request(D, dtype, x_req, W, r, yr.data());
+  bool same = true;
+  for (int64_t k = 0; k < D.o_r * D.d; ++k) same = same && (Y[(size_t)k] == yr[(size_t)k]);
+  for (int64_t o = 0; o < D.o_c; ++o)
+    for (int64_t c = 0; c < D.d; ++c) y_cand[o * D.d + c] = Y[(size_t)((D.o_r + o) * D.d + c)];
+  return same;
+}
+
+// ---- DCA, one candidate: Eq. (13) with the K/V broadcast materialised ------------------
+struct DcaDims {
+  int64_t q, H, dh;
+  double scale;
+};
+
+// o [q x H x dh], lse [q x H] for candidate i of request r with keys [s0, s1)
+void dca_candidate(const DcaDims& D, const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t i, int64_t s0,
+                   int64_t s1, const double* q_override /* [q x H x dh] or null */, double* o, double* lse) {
+  const int64_t L = s1 - s0, row = D.H * D.dh;
+  // the explicit broadcast: fresh per-candidate copies of the request's K and V
+  std::vector<double> Ki((size_t)(L * row)), Vi((size_t)(L * row));
+  for (int64_t j = 0; j < L; ++j)
+    for (int64_t e = 0; e < row; ++e) {
+      Ki[(size_t)(j * row + e)] = widen(K, 1, (s0 + j) * row + e);
+      Vi[(size_t)(j * row + e)] = widen(V, 1, (s0 + j) * row + e);
+    }
+  std::vector<double> s((size_t)L), p((size_t)L);
+  for (int64_t t = 0; t < D.q; ++t)
+    for (int64_t h = 0; h < D.H; ++h) {
+      double* out = o + (t * D.H + h) * D.dh;
+      if (L == 0) {  // empty key sequence: zero output, LSE = -inf
+        for (int64_t c = 0; c < D.dh; ++c) out[c] = 0.0;
+        lse[t * D.H + h] = -std::numeric_limits<double>::infinity();
+        continue;
+      }
+      double m = -std::numeric_limits<double>::infinity();
+      for (int64_t j = 0; j < L; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < D.dh; ++c) {
+          const double qv = q_override ? q_override[(t * D.H + h) * D.dh + c]
+                                       : widen(Q, 1, ((i * D.q + t) * D.H + h) * D.dh + c);
+          acc += qv * Ki[(size_t)(j * row + h * D.dh + c)];
+        }
+        s[(size_t)j] = D.scale * acc;
+        if (s[(size_t)j] > m) m = s[(size_t)j];
+      }
+      double l = 0.0;
+      for (int64_t j = 0; j < L; ++j) {
+        p[(size_t)j] = std::exp(s[(size_t)j] - m);
+        l += p[(size_t)j];
+      }
+      for (int64_t c = 0; c < D.dh; ++c) out[c] = 0.0;
+      for (int64_t j = 0; j < L; ++j) {
+        const double w = p[(size_t)j] / l;
+        for (int64_t c = 0; c < D.dh; ++c) out[c] += w * Vi[(size_t)(j * row + h * D.dh + c)];
+      }
+      lse[t * D.H + h] = m + std::log(l);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int rocs_oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+// IKBO-LCB oracle.  dtype 0 = fp32 inputs, 1 = bf16 inputs (bit patterns).
+// Computes Y^R for the requests listed in sel_req (y_req: [n_sel_req, o_r, d]) and
+// Y^C for the candidates listed in sel_cand (y_cand: [n_sel_cand, o_c, d]).
+int rocs_oracle_lcb(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n_c, int64_t d, int64_t o_r, int64_t o_c,
+                    int dtype, const void* x_req, const void* x_cand, const void* w_rr, const void* w_cr,
+                    const void* w_cc, int64_t n_sel_req, const int64_t* sel_req, double* y_req, int64_t n_sel_cand,
+                    const int64_t* sel_cand, double* y_cand, int nthreads) {
+  if (n_r < 0 || n_c < 0 || d < 0 || o_r < 0 || o_c < 0 || (dtype != 0 && dtype != 1)) return ORC_INVALID;
+  if (!csr_ok(cand_off, R, -1)) return ORC_BAD_OFFSETS;
+  set_threads(nthreads);
+  const LcbDims D{n_r, n_c, d, o_r, o_c};
+  const int64_t C = cand_off[R];
+  std::vector<int64_t> m = index_map(cand_off, R);
+  std::vector<double> W;
+  lcb_full_weight(D, dtype, w_rr, w_cr, w_cc, W);
+  for (int64_t k = 0; k < n_sel_req; ++k)
+    if (sel_req[k] < 0 || sel_req[k] >= R) return ORC_INVALID;
+  for (int64_t k = 0; k < n_sel_cand; ++k)
+    if (sel_cand[k] < 0 || sel_cand[k] >= C) return ORC_INVALID;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t k = 0; k < n_sel_req; ++k) lcb_request(D, dtype, x_req, W, sel_req[k], y_req + k * o_r * d);
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t k = 0; k < n_sel_cand; ++k) {
+    const int64_t i = sel_cand[k];
+    if (!lcb_candidate(D, dtype, x_req, x_cand, W, i, m[(size_t)i], y_cand + k * o_c * d)) bad |= 1;
+  }
+  return bad ? ORC_ISOLATION : ORC_OK;
+}
+
+// IKBO-DCA oracle for the candidates in sel_cand: o [n_sel, q, H, dh], lse [n_sel, q, H].
+int rocs_oracle_dca(int64_t R, const int32_t* cand_off, const int32_t* seq_off, int64_t q, int64_t H, int64_t dh,
+                    double scale, const uint16_t* Q, const uint16_t* K, const uint16_t* V, int64_t n_sel,
+                    const int64_t* sel_cand, double* o, double* lse, int nthreads) {
+  if (q < 0 || H < 0 || dh < 0) return ORC_INVALID;
+  if (!csr_ok(cand_off, R, -1) || !csr_ok(seq_off, R, -1)) return ORC_BAD_OFFSETS;
+  set_threads(nthreads);
+  const int64_t C = cand_off[R];
+  for (int64_t k = 0; k < n_sel; ++k)
+    if (sel_cand[k] < 0 || sel_cand[k] >= C) return ORC_INVALID;
+  std::vector<int64_t> m = index_map(cand_off, R);
+  const DcaDims D{q, H, dh, scale};
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t k = 0; k < n_sel; ++k) {
+    const int64_t i = sel_cand[k], r = m[(size_t)i];
+    dca_candidate(D, Q, K, V, i, seq_off[r], seq_off[r + 1], nullptr, o + k * q * H * dh, lse + k * q * H);
+  }
+  return ORC_OK;
+}
+
+// Linear query projection: q_out[k, n] = sum_j w_q[n, j] * y[k, j], j ascending.
+// y is bf16 bit patterns [n_rows, n_in]; w_q bf16 [n_out, n_in]; q_out double [n_rows, n_out].
+int rocs_oracle_proj(int64_t n_rows, int64_t n_in, int64_t n_out, const uint16_t* y, const uint16_t* w_q,
+                     double* q_out, int nthreads) {
+  if (n_rows < 0 || n_in < 0 || n_out < 0) return ORC_INVALID;
+  set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t k = 0; k < n_rows; ++k)
+    for (int64_t n = 0; n < n_out; ++n) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < n_in; ++j) acc += widen(w_q, 1, n * n_in + j) * widen(y, 1, k * n_in + j);
+      q_out[k * n_out + n] = acc;
+    }
+  return ORC_OK;
+}
+
+// Chained block for the candidates in sel_cand (q = 1 query token per candidate):
+//   Y^C_i (LCB, Eq. 6) -> round to bf16 -> Q_i = W_q . vec(Y^C_i) -> round to bf16
+//   -> DCA over request m_i's keys with H heads of size dh.
+// Outputs: y_cand [n_sel, o_c, d] (before rounding), q_out [n_sel, H*dh] (before rounding),
+// o [n_sel, H, dh], lse [n_sel, H].
+int rocs_oracle_chain(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n_c, int64_t d, int64_t o_r,
+                      int64_t o_c, const uint16_t* x_req, const uint16_t* x_cand, const uint16_t* w_rr,
+                      const uint16_t* w_cr, const uint16_t* w_cc, const uint16_t* w_q, const int32_t* seq_off,
+                      int64_t H, int64_t dh, double scale, const uint16_t* K, const uint16_t* V, int64_t n_sel,
+                      const int64_t* sel_cand, double* y_cand, double* q_out, double* o, double* lse, int nthreads) {
+  if (!csr_ok(cand_off, R, -1) || !csr_ok(seq_off, R, -1)) return ORC_BAD_OFFSETS;
+  set_threads(nthreads);
+  const LcbDims D{n_r, n_c, d, o_r, o_c};
+  const int64_t C = cand_off[R], n_in = o_c * d, n_out = H * dh;
+  for (int64_t k = 0; k < n_sel; ++k)
+    if (sel_cand[k] < 0 || sel_cand[k] >= C) return ORC_INVALID;
+  std::vector<int64_t> m = index_map(cand_off, R);
+  std::vector<double> W;
+  lcb_full_weight(D, 1, w_rr, w_cr, w_cc, W);
+  const DcaDims DD{1, H, dh, scale};
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t k = 0; k < n_sel; ++k) {
+    const int64_t i = sel_cand[k], r = m[(size_t)i];
+    double* yc = y_cand + k * n_in;
+    if (!lcb_candidate(D, 1, x_req, x_cand, W, i, r, yc)) bad |= 1;
+    std::vector<double> yb((size_t)n_in), qb((size_t)n_out);
+    for (int64_t j = 0; j < n_in; ++j) yb[(size_t)j] = round_bf16(yc[j]);
+    for (int64_t n = 0; n < n_out; ++n) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < n_in; ++j) acc += widen(w_q, 1, n * n_in + j) * yb[(size_t)j];
+      q_out[k * n_out + n] = acc;
+      qb[(size_t)n] = round_bf16(acc);
+    }
+    dca_candidate(DD, nullptr, K, V, i, seq_off[r], seq_off[r + 1], qb.data(), o + k * n_out, lse + k * H);
+  }
+  return bad ? ORC_ISOLATION : ORC_OK;
+}
+
+// Exposed for the oracle's own tests of its bf16 rounding.
+double rocs_oracle_round_bf16(double x) { return round_bf16(x); }
+
+}  // extern "C"

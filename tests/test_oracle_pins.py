@@ -1,0 +1,376 @@
+"""Pins for the fp64 oracle, each against something other than the oracle itself.
+
+Sources (ROCS, arXiv:2607.27744, paper-archivist reading notes):
+  Eq. (1)/(2)/(11)  GLM isolation and request-output identity   (section 3.1.1, 3.1.5)
+  Eq. (5)/(6)       ROCSified LCB, two-group form              (section 3.1.2)
+  Eq. (14)          IKBO decomposition Z = W_CR X^R, Y^C = Z_m + W_CC X^C  (section 4.1)
+  Eq. (13)          group-wise cross attention                 (section 3.2)
+A planted mistake in the oracle (dropped term, wrong sign/index, transposed
+operand, missing max-subtraction or normalisation) fails at least one of these.
+"""
+import math
+import os
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import rocs_inputs as ri
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_golden(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, *vals = line.split()
+            out[k] = [float(v) for v in vals]
+    return out
+
+
+def _f32(a):
+    return np.asarray(a, dtype=np.float32)
+
+
+def _bf16_exact(a):
+    """float values exactly representable in bf16 -> bit patterns."""
+    f = np.asarray(a, dtype=np.float32)
+    b = (f.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(ri.bf16_to_f32(b), f), "value not exact in bf16"
+    return b
+
+
+def _w(x):
+    return x if x.dtype == np.float32 else ri.bf16_to_f32(x)
+
+
+def _rand_lcb(seed, counts, n_r=5, n_c=3, d=7, o_r=4, o_c=6, dtype="f32"):
+    return ri.make_lcb("t", counts, n_r, n_c, d, o_r, o_c, seed, dtype)
+
+
+# ------------------------------------------------------------------------------ LCB
+def test_lcb_golden_two_group(oracle_mod):
+    g = _read_golden("lcb_two_group.txt")
+    for conv in (_f32, _bf16_exact):
+        x_req = conv(np.array(g["x_req"]).reshape(1, 2, 2))
+        x_cand = conv(np.array(g["x_cand"]).reshape(2, 2, 2))
+        w_rr, w_cr, w_cc = (conv(np.array(g[k]).reshape(1, 2)) for k in ("w_rr", "w_cr", "w_cc"))
+        yr, yc = oracle_mod.lcb([0, 2], x_req, x_cand, w_rr, w_cr, w_cc)
+        assert yr.ravel().tolist() == g["y_req"]
+        assert yc.ravel().tolist() == g["y_cand"]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_lcb_bruteforce_group_sum(oracle_mod, dtype):
+    """Eq. (5): Y^(i) = sum_{j<=i} W_ij X^(j), evaluated element by element with exact
+    rational arithmetic over the group loop (group 0 = request, group 1 = candidate)."""
+    x = _rand_lcb(11, [2, 0, 3], dtype=dtype)
+    yr, yc = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)
+    XR, XC = _w(x.x_req).astype(np.float64), _w(x.x_cand).astype(np.float64)
+    W = {(0, 0): _w(x.w_rr), (1, 0): _w(x.w_cr), (1, 1): _w(x.w_cc)}
+    m = [r for r in range(x.R) for _ in range(x.cand_off[r], x.cand_off[r + 1])]
+    for r in range(x.R):
+        for o in range(x.o_r):
+            for c in range(x.d):
+                exact = sum(Fraction(float(W[0, 0][o, k])) * Fraction(XR[r, k, c]) for k in range(x.n_r))
+                assert abs(yr[r, o, c] - float(exact)) <= 1e-12 * (1 + abs(float(exact)))
+    for i in range(x.C):
+        groups = [XR[m[i]], XC[i]]
+        for o in range(x.o_c):
+            for c in range(x.d):
+                exact = Fraction(0)
+                for j in range(0, 2):  # j <= i for output group i = 1
+                    Wij = W[1, j]
+                    for k in range(Wij.shape[1]):
+                        exact += Fraction(float(Wij[o, k])) * Fraction(groups[j][k, c])
+                assert abs(yc[i, o, c] - float(exact)) <= 1e-12 * (1 + abs(float(exact)))
+
+
+def test_lcb_decomposition_eq14(oracle_mod):
+    """IKBO decomposition (Eq. 14) computed with library matmuls equals the materialised Eq. (6)."""
+    x = _rand_lcb(5, [4, 1, 0, 6], n_r=9, n_c=5, d=16, o_r=8, o_c=12)
+    yr, yc = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)
+    XR, XC = _w(x.x_req).astype(np.float64), _w(x.x_cand).astype(np.float64)
+    WRR, WCR, WCC = (_w(a).astype(np.float64) for a in (x.w_rr, x.w_cr, x.w_cc))
+    stacked = np.concatenate([WRR, WCR], axis=0)  # [W_RR; W_CR] . X^R in one GEMM at batch B_r
+    YZ = np.einsum("on,rnd->rod", stacked, XR)
+    Y_R, Z = YZ[:, : x.o_r], YZ[:, x.o_r:]
+    m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+    Y_C = Z[m] + np.einsum("on,ind->iod", WCC, XC)
+    scale = np.abs(Y_C).max()
+    assert np.abs(yr - Y_R).max() <= 1e-12 * np.abs(Y_R).max()
+    assert np.abs(yc - Y_C).max() <= 1e-12 * scale
+
+
+def test_lcb_isolation_bitwise(oracle_mod):
+    """Eq. (1)/(2): request outputs do not depend on candidate inputs, bit for bit;
+    and a candidate's output does not depend on other candidates."""
+    x = _rand_lcb(7, [3, 5], n_r=6, n_c=4, d=8, o_r=5, o_c=5)
+    yr0, yc0 = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)
+    x2 = ri.normal(99, 1, x.x_cand.shape, 3.0, "f32")
+    yr1, yc1 = oracle_mod.lcb(x.cand_off, x.x_req, x2, x.w_rr, x.w_cr, x.w_cc)
+    assert np.array_equal(yr0, yr1)
+    assert not np.array_equal(yc0, yc1)
+    x3 = x.x_cand.copy()
+    x3[4] += 1.0  # perturb candidate 4 only
+    _, yc3 = oracle_mod.lcb(x.cand_off, x.x_req, x3, x.w_rr, x.w_cr, x.w_cc)
+    keep = [i for i in range(x.C) if i != 4]
+    assert np.array_equal(yc0[keep], yc3[keep]) and not np.array_equal(yc0[4], yc3[4])
+
+
+def test_lcb_permutation_within_request(oracle_mod):
+    x = _rand_lcb(8, [5, 4], n_r=4, n_c=4, d=8)
+    perm = np.array([3, 0, 4, 1, 2, 8, 6, 5, 7])
+    _, yc0 = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)
+    _, yc1 = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand[perm], x.w_rr, x.w_cr, x.w_cc)
+    assert np.array_equal(yc1, yc0[perm])
+
+
+def test_lcb_closed_forms(oracle_mod):
+    x = _rand_lcb(9, [2, 3], n_r=6, n_c=5, d=4, o_r=3, o_c=4)
+    XR, XC = _w(x.x_req).astype(np.float64), _w(x.x_cand).astype(np.float64)
+    m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+    WCR, WCC = _w(x.w_cr).astype(np.float64), _w(x.w_cc).astype(np.float64)
+    # W_CC = 0  ->  Y^C_i = W_CR X^R_{m_i}
+    _, yc = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, np.zeros_like(x.w_cc))
+    np.testing.assert_allclose(yc, (WCR @ XR)[m], rtol=1e-12, atol=1e-12)
+    # W_CR = 0  ->  Y^C_i = W_CC X^C_i
+    _, yc = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, np.zeros_like(x.w_cr), x.w_cc)
+    np.testing.assert_allclose(yc, WCC @ XC, rtol=1e-12, atol=1e-12)
+    # one request -> a textbook GEMM [W_CR W_CC] . [X^R ; X^C_i]
+    x1 = _rand_lcb(10, [4], n_r=6, n_c=5, d=4, o_r=3, o_c=4)
+    _, yc = oracle_mod.lcb(x1.cand_off, x1.x_req, x1.x_cand, x1.w_rr, x1.w_cr, x1.w_cc)
+    Wcat = np.concatenate([_w(x1.w_cr), _w(x1.w_cc)], axis=1).astype(np.float64)
+    for i in range(4):
+        Xcat = np.concatenate([_w(x1.x_req)[0], _w(x1.x_cand)[i]], axis=0).astype(np.float64)
+        np.testing.assert_allclose(yc[i], Wcat @ Xcat, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_lcb_index_probe_exact(oracle_mod, dtype):
+    """W_CC = 0, W_CR selects input row 0, X^R_r == r  ->  Y^C_i == m_i exactly."""
+    counts = [3, 0, 4, 1, 0, 2]
+    x = _rand_lcb(12, counts, n_r=4, n_c=3, d=5, o_r=2, o_c=3, dtype=dtype)
+    conv = _f32 if dtype == "f32" else _bf16_exact
+    x_req = conv(np.broadcast_to(np.arange(x.R, dtype=np.float32)[:, None, None], x.x_req.shape))
+    w_cr = np.zeros((x.o_c, x.n_r), np.float32)
+    w_cr[:, 0] = 1.0
+    _, yc = oracle_mod.lcb(x.cand_off, x_req, x.x_cand, x.w_rr, conv(w_cr), conv(np.zeros((x.o_c, x.n_c))))
+    m = np.repeat(np.arange(x.R), counts)
+    assert np.array_equal(yc, np.broadcast_to(m[:, None, None].astype(np.float64), yc.shape))
+
+
+def test_lcb_selection_and_bad_offsets(oracle_mod):
+    x = _rand_lcb(13, [2, 3, 1])
+    yr, yc = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)
+    yr2, yc2 = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, sel_req=[2, 0],
+                              sel_cand=[5, 1])
+    assert np.array_equal(yr2, yr[[2, 0]]) and np.array_equal(yc2, yc[[5, 1]])
+    with pytest.raises(oracle_mod.OracleError) as e:
+        oracle_mod.lcb(np.array([0, 3, 2, 6]), x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)
+    assert e.value.code == oracle_mod.ORC_BAD_OFFSETS
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.lcb(np.array([1, 3, 5, 6]), x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)
+
+
+# ------------------------------------------------------------------------------ DCA
+def _dca_inputs(seed, counts, lengths, q=2, H=2, dh=8):
+    return ri.make_dca("t", counts, lengths, q, H, dh, seed)
+
+
+def test_dca_golden(oracle_mod):
+    g = _read_golden("dca_softmax.txt")
+    for case in ("case1", "case2"):
+        k = np.array(g[f"{case}_k"])
+        L = len(k)
+        o, lse = oracle_mod.dca([0, 1], [0, L], _bf16_exact(np.array(g[f"{case}_q"]).reshape(1, 1, 1)),
+                                _bf16_exact(k.reshape(L, 1, 1)), _bf16_exact(np.array(g[f"{case}_v"]).reshape(L, 1, 1)),
+                                q=1, scale=g[f"{case}_scale"][0])
+        assert abs(o.item() - g[f"{case}_o"][0]) <= 1e-12
+        assert abs(lse.item() - g[f"{case}_lse"][0]) <= 1e-12
+
+
+def test_dca_bruteforce_decimal(oracle_mod):
+    """Naive softmax attention in 40-digit decimal arithmetic (exact inputs)."""
+    getcontext().prec = 40
+    x = _dca_inputs(21, [2, 1, 0], [5, 3, 2], q=2, H=2, dh=4)
+    o, lse = oracle_mod.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, x.v_t, x.q, x.scale)
+    Q, K, V = (ri.bf16_to_f32(a).astype(np.float64) for a in (x.q_t, x.k_t, x.v_t))
+    sc = Decimal(x.scale)
+    m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+    for i in range(x.C):
+        r = m[i]
+        s0, s1 = x.seq_off[r], x.seq_off[r + 1]
+        for t in range(x.q):
+            for h in range(x.H):
+                qv = [Decimal(float(v)) for v in Q[i * x.q + t, h]]
+                s = [sc * sum(qv[c] * Decimal(float(K[j, h, c])) for c in range(x.dh)) for j in range(s0, s1)]
+                e = [v.exp() for v in s]
+                den = sum(e)
+                for c in range(x.dh):
+                    ref = sum(e[j] * Decimal(float(V[s0 + j, h, c])) for j in range(s1 - s0)) / den
+                    assert abs(o[i, t, h, c] - float(ref)) <= 1e-12
+                assert abs(lse[i, t, h] - float(den.ln())) <= 1e-12
+
+
+def test_dca_matches_library_attention(oracle_mod):
+    """Per request, DCA is plain non-causal attention of all its candidates' query rows over
+    that request's K/V: torch's scaled_dot_product_attention in float64."""
+    x = _dca_inputs(22, [3, 2, 4], [17, 9, 33], q=3, H=3, dh=16)
+    o, _ = oracle_mod.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, x.v_t, x.q, x.scale)
+    Q, K, V = (torch.from_numpy(ri.bf16_to_f32(a).astype(np.float64)) for a in (x.q_t, x.k_t, x.v_t))
+    for r in range(x.R):
+        rows = slice(x.q * x.cand_off[r], x.q * x.cand_off[r + 1])
+        keys = slice(x.seq_off[r], x.seq_off[r + 1])
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            Q[rows].transpose(0, 1), K[keys].transpose(0, 1), V[keys].transpose(0, 1), scale=x.scale)
+        got = torch.from_numpy(o[x.cand_off[r]: x.cand_off[r + 1]].reshape(-1, x.H, x.dh)).transpose(0, 1)
+        assert torch.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_dca_rows_sum_to_one(oracle_mod):
+    """V = one-hot basis (L <= dh): O[:, c] is softmax weight c, so each row sums to 1 and is >= 0."""
+    L, dh = 6, 8
+    x = _dca_inputs(23, [3], [L], q=2, H=2, dh=dh)
+    v = np.zeros((L, 2, dh), np.float32)
+    for j in range(L):
+        v[j, :, j] = 1.0
+    o, _ = oracle_mod.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, _bf16_exact(v), x.q, x.scale)
+    assert np.all(o >= 0) and np.all(o[..., L:] == 0)
+    assert np.abs(o.sum(-1) - 1.0).max() <= 1e-12
+
+
+def test_dca_closed_forms(oracle_mod):
+    x = _dca_inputs(24, [2, 2], [7, 1], q=1, H=1, dh=4)
+    Vf = ri.bf16_to_f32(x.v_t).astype(np.float64)
+    # all V rows equal -> O = v
+    vconst = np.broadcast_to(np.array([1.5, -2.0, 0.25, 3.0], np.float32), x.v_t.shape)
+    o, _ = oracle_mod.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, _bf16_exact(vconst), 1, x.scale)
+    assert np.abs(o - vconst[0, 0]).max() <= 1e-12
+    # all K rows equal (zero) -> uniform weights -> O = mean(V_r), LSE = log L_r
+    o, lse = oracle_mod.dca(x.cand_off, x.seq_off, x.q_t, np.zeros_like(x.k_t), x.v_t, 1, x.scale)
+    assert np.abs(o[0, 0, 0] - Vf[0:7, 0].mean(0)).max() <= 1e-12
+    assert abs(lse[0, 0, 0] - math.log(7)) <= 1e-12
+    # L_r = 1 -> O = V_0 of that request
+    assert np.abs(o[2, 0, 0] - Vf[7, 0]).max() <= 1e-12
+    assert abs(lse[2, 0, 0] - 0.0) <= 1e-12
+    # one dominant score -> O ~ that V row
+    k = np.zeros((8, 1, 4), np.float32)
+    k[3, 0, 0] = 64.0
+    qv = np.zeros((4, 1, 4), np.float32)
+    qv[:, 0, 0] = 1.0
+    o, _ = oracle_mod.dca(x.cand_off, x.seq_off, _bf16_exact(qv), _bf16_exact(k), x.v_t, 1, 1.0)
+    # p_3 = 1 / (1 + 7 e^-64): O equals V_3 far below double precision
+    assert np.abs(o[0, 0, 0] - Vf[3, 0]).max() <= 1e-12
+
+
+def test_dca_index_probe_and_empty(oracle_mod):
+    counts, lengths = [2, 3, 1, 2], [4, 0, 2, 5]
+    x = _dca_inputs(25, counts, lengths, q=2, H=2, dh=4)
+    v = np.zeros(x.v_t.shape, np.float32)
+    for r in range(x.R):
+        v[x.seq_off[r]: x.seq_off[r + 1]] = r
+    o, lse = oracle_mod.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, _bf16_exact(v), x.q, x.scale)
+    m = np.repeat(np.arange(x.R), counts)
+    for i in range(x.C):
+        if lengths[m[i]] == 0:
+            assert np.all(o[i] == 0) and np.all(np.isneginf(lse[i]))
+        else:
+            assert np.abs(o[i] - m[i]).max() <= 1e-12
+
+
+def test_dca_permutation_within_request(oracle_mod):
+    x = _dca_inputs(26, [4, 3], [6, 9], q=2, H=2, dh=8)
+    o0, l0 = oracle_mod.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, x.v_t, x.q, x.scale)
+    perm = np.array([2, 0, 3, 1, 6, 4, 5])
+    qp = x.q_t.reshape(x.C, x.q, x.H, x.dh)[perm].reshape(x.q_t.shape)
+    o1, l1 = oracle_mod.dca(x.cand_off, x.seq_off, qp, x.k_t, x.v_t, x.q, x.scale)
+    assert np.array_equal(o1, o0[perm]) and np.array_equal(l1, l0[perm])
+
+
+# ------------------------------------------------------------------------------ projection / chain
+def test_round_bf16(oracle_mod):
+    rb = oracle_mod.round_bf16
+    one = 1.0
+    assert rb(one + 2 ** -8) == one  # tie -> even
+    assert rb(one + 3 * 2 ** -8) == one + 2 ** -6  # tie -> even (up)
+    assert rb(one + 2 ** -8 + 2 ** -30) == one + 2 ** -7  # above the tie
+    assert rb(-(one + 2 ** -8 + 2 ** -30)) == -(one + 2 ** -7)
+    assert rb(2 ** -133 * 0.75) == 2 ** -133  # subnormal quantum
+    assert rb(2.0 ** 128 * 0.999999) == math.inf
+    # values exactly representable in fp32: agree with the fp32 -> bf16 RNE bit rule
+    f = ri.normal(3, 9, (2000,), 10.0, "f32")
+    u = f.view(np.uint32).astype(np.uint64)
+    bits = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    ref = ri.bf16_to_f32(bits).astype(np.float64)
+    got = np.array([rb(float(v)) for v in f])
+    assert np.array_equal(got, ref)
+
+
+def test_proj_matches_library_matmul(oracle_mod):
+    y = ri.normal(31, 1, (5, 96))
+    w = ri.normal(31, 2, (24, 96), 0.1)
+    got = oracle_mod.proj(y, w)
+    ref = ri.bf16_to_f32(y).astype(np.float64) @ ri.bf16_to_f32(w).astype(np.float64).T
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def _small_chain(seed=41):
+    return ri.chain(seed=seed, R=3, median=3, sigma=0.5, clip=(1, 6), Llo=1, Lhi=9, H=2, dh=8)
+
+
+def _shrink_chain(ci):
+    """shrink the LCB to n_r=8, n_c=4, d=4, o_r=4, o_c=4 so the oracle runs in milliseconds."""
+    counts = np.diff(ci.lcb.cand_off)
+    ci.lcb = ri.make_lcb("t", counts, 8, 4, 4, 4, 4, 41)
+    ci.w_q = ri.normal(41, ri.S_WQ, (ci.H * ci.dh, 16), 0.25)
+    return ci
+
+
+def test_chain_composes_stages(oracle_mod):
+    ci = _shrink_chain(_small_chain())
+    x = ci.lcb
+    sel = np.arange(x.C)
+    y, qo, o, lse = oracle_mod.chain(ci, sel)
+    _, yc = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)
+    assert np.array_equal(y, yc)
+    yb = np.array([[oracle_mod.round_bf16(v) for v in row] for row in yc.reshape(x.C, -1)])
+    ybits = (yb.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    qref = oracle_mod.proj(ybits, ci.w_q)
+    assert np.array_equal(qo, qref)
+    qb = np.array([[oracle_mod.round_bf16(v) for v in row] for row in qref])
+    qbits = (qb.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16).reshape(x.C, ci.H, ci.dh)
+    o2, l2 = oracle_mod.dca(x.cand_off, ci.seq_off, qbits, ci.k_t, ci.v_t, 1, ci.scale)
+    assert np.array_equal(o, o2[:, 0]) and np.array_equal(lse, l2[:, 0])
+
+
+def test_chain_zero_projection(oracle_mod):
+    """W_q = 0 -> every query is 0 -> uniform attention -> O = mean of the request's V rows."""
+    ci = _shrink_chain(_small_chain(43))
+    ci.w_q = np.zeros_like(ci.w_q)
+    x = ci.lcb
+    _, qo, o, _ = oracle_mod.chain(ci, np.arange(x.C))
+    assert np.all(qo == 0)
+    V = ri.bf16_to_f32(ci.v_t).astype(np.float64)
+    m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+    for i in range(x.C):
+        s0, s1 = ci.seq_off[m[i]], ci.seq_off[m[i] + 1]
+        assert np.abs(o[i] - V[s0:s1].mean(0)).max() <= 1e-12
+
+
+def test_dca_large_scores_stable(oracle_mod):
+    """Scores 800 and 796 (exp overflows double without the max shift): weights are
+    sigma(4) and 1 - sigma(4) exactly as the softmax definition gives."""
+    q = _bf16_exact(np.array([1.0]).reshape(1, 1, 1))
+    k = _bf16_exact(np.array([800.0, 796.0]).reshape(2, 1, 1))
+    v = _bf16_exact(np.array([1.0, 0.0]).reshape(2, 1, 1))
+    o, lse = oracle_mod.dca([0, 1], [0, 2], q, k, v, q=1, scale=1.0)
+    w0 = 1.0 / (1.0 + math.exp(-4.0))
+    assert abs(o.item() - w0) <= 1e-12
+    assert abs(lse.item() - (800.0 + math.log1p(math.exp(-4.0)))) <= 1e-12
