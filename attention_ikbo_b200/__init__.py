@@ -1,0 +1,31 @@
+"""B200 (sm_100a) In-Kernel Broadcast Optimization: IKBO-LCB and IKBO-DCA.
+
+Thin Python binding over the C ABI in ``include/rocs_ikbo.h`` (``librocs_ikbo.so``).
+Every step of the computation runs in the library's CUDA kernels; this module only
+marshals torch tensors (device memory, streams) into the C argument structs.  There is
+no CPU or PyTorch fallback: if the native library is missing, importing the binding
+functions raises.
+
+Operations ("ROCS: Request-Oriented Compute Sharing ...", arXiv:2607.27744):
+  * :func:`rocs_lcb_forward` -- section 3.1.2 Eq. (6) via the section 4.1 Eq. (14)
+    decomposition, broadcast-add fused into the candidate GEMM epilogue (section 4.2).
+  * :func:`rocs_dca_forward` -- section 3.2 Eq. (13) candidate cross attention over K/V
+    stored once per request (section 4.3).
+  * :func:`rocs_proj_forward` -- linear query projection of the chained block (Eq. 12).
+"""
+from ._binding import (  # noqa: F401
+    ROCS_BF16,
+    ROCS_F32,
+    RocsError,
+    chain_forward,
+    last_launch_count,
+    lib_path,
+    load_library,
+    rocs_dca_forward,
+    rocs_dca_forward_expand,
+    rocs_lcb_forward,
+    rocs_lcb_forward_expand,
+    rocs_proj_forward,
+    rocs_read_status,
+    STATUS_NAMES,
+)

@@ -1,0 +1,256 @@
+"""ctypes marshalling for ``librocs_ikbo.so`` (see ``include/rocs_ikbo.h`` for the contract)."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "librocs_ikbo.so")
+
+ROCS_F32, ROCS_BF16 = 0, 1
+STATUS_NAMES = {0: "ROCS_OK", 1: "ROCS_ERR_INVALID_ARG", 2: "ROCS_ERR_BAD_OFFSETS", 3: "ROCS_ERR_UNSUPPORTED",
+                4: "ROCS_ERR_CUDA", 5: "ROCS_ERR_TIMEOUT", 6: "ROCS_ERR_WORKSPACE", 7: "ROCS_ERR_DEVICE_INDEX"}
+
+_i64, _i32, _vp, _f32, _sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+
+
+class RocsError(RuntimeError):
+    def __init__(self, code, what=""):
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class LcbArgs(ctypes.Structure):
+    _fields_ = [("R", _i64), ("n_r", _i64), ("n_c", _i64), ("d", _i64), ("o_r", _i64), ("o_c", _i64),
+                ("dtype", _i32), ("cand_off_dev", _vp), ("cand_off_host", _vp), ("x_req", _vp), ("x_cand", _vp),
+                ("w_rr", _vp), ("w_cr", _vp), ("w_cc", _vp), ("y_req", _vp), ("y_cand", _vp),
+                ("workspace", _vp), ("workspace_bytes", _sz)]
+
+
+class DcaArgs(ctypes.Structure):
+    _fields_ = [("R", _i64), ("q", _i64), ("H", _i64), ("dh", _i64), ("scale", _f32),
+                ("cand_off_dev", _vp), ("cand_off_host", _vp), ("seq_off_dev", _vp), ("seq_off_host", _vp),
+                ("q_ptr", _vp), ("k_ptr", _vp), ("v_ptr", _vp), ("o_ptr", _vp), ("lse_ptr", _vp),
+                ("workspace", _vp), ("workspace_bytes", _sz)]
+
+
+class ProjArgs(ctypes.Structure):
+    _fields_ = [("M", _i64), ("N", _i64), ("K", _i64), ("in_", _vp), ("w", _vp), ("out", _vp),
+                ("workspace", _vp), ("workspace_bytes", _sz)]
+
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load the native library; raises if it has not been built (no fallback path exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m attention_ikbo_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.POINTER
+        for name, argt in [("rocs_lcb_workspace_size", [P(LcbArgs)]), ("rocs_lcb_expand_workspace_size", [P(LcbArgs)]),
+                           ("rocs_dca_workspace_size", [P(DcaArgs)]), ("rocs_proj_workspace_size", [P(ProjArgs)]),
+                           ("rocs_dca_expand_workspace_size", [P(DcaArgs), _i64])]:
+            getattr(lib, name).restype = _sz
+            getattr(lib, name).argtypes = argt
+        for name, argt in [("rocs_lcb_forward", [P(LcbArgs), _vp]), ("rocs_lcb_forward_expand", [P(LcbArgs), _vp]),
+                           ("rocs_dca_forward", [P(DcaArgs), _vp]), ("rocs_proj_forward", [P(ProjArgs), _vp]),
+                           ("rocs_dca_forward_expand", [P(DcaArgs), _i64, _vp]),
+                           ("rocs_read_status", [_vp, _vp, P(_i32), P(_i32)])]:
+            getattr(lib, name).restype = ctypes.c_int
+            getattr(lib, name).argtypes = argt
+        lib.rocs_status_string.restype = ctypes.c_char_p
+        lib.rocs_status_string.argtypes = [ctypes.c_int]
+        lib.rocs_last_launch_count.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def last_launch_count() -> int:
+    """Kernel launches enqueued by the last successful forward call on this thread."""
+    return int(load_library().rocs_last_launch_count())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _offsets(off, device):
+    """(device int32 tensor, host int32 numpy array) from a tensor / array / list."""
+    if isinstance(off, torch.Tensor):
+        host = off.detach().to("cpu", torch.int32).contiguous().numpy()
+        dev = off if (off.is_cuda and off.dtype == torch.int32 and off.is_contiguous()) else \
+            torch.from_numpy(host).to(device)
+    else:
+        host = np.ascontiguousarray(np.asarray(off, dtype=np.int32))
+        dev = torch.from_numpy(host).to(device)
+    return dev, host
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise RocsError(rc, what)
+
+
+def _workspace(nbytes, device, given):
+    if given is not None:
+        if given.numel() * given.element_size() < nbytes:
+            raise RocsError(6, "workspace")
+        return given
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y_cand):
+    dev = x_req.device
+    dtype = {torch.float32: ROCS_F32, torch.bfloat16: ROCS_BF16}[x_req.dtype]
+    off_d, off_h = _offsets(cand_off, dev)
+    R, n_r, d = x_req.shape
+    C = int(off_h[-1])
+    n_c, o_r, o_c = x_cand.shape[1] if x_cand.dim() == 3 else w_cc.shape[1], w_rr.shape[0], w_cc.shape[0]
+    if y_req is None:
+        y_req = torch.empty((R, o_r, d), dtype=x_req.dtype, device=dev)
+    if y_cand is None:
+        y_cand = torch.empty((C, o_c, d), dtype=x_req.dtype, device=dev)
+    for t in (x_req, x_cand, w_rr, w_cr, w_cc, y_req, y_cand):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == x_req.dtype):
+            raise RocsError(1, "LCB tensors must be contiguous CUDA tensors of one dtype")
+    a = LcbArgs(R=R, n_r=n_r, n_c=n_c, d=d, o_r=o_r, o_c=o_c, dtype=dtype,
+                cand_off_dev=off_d.data_ptr(), cand_off_host=off_h.ctypes.data,
+                x_req=x_req.data_ptr(), x_cand=x_cand.data_ptr() if C else None, w_rr=w_rr.data_ptr(),
+                w_cr=w_cr.data_ptr(), w_cc=w_cc.data_ptr(), y_req=y_req.data_ptr(),
+                y_cand=y_cand.data_ptr() if C else None)
+    return a, (off_d, off_h), y_req, y_cand
+
+
+def rocs_lcb_forward(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req=None, y_cand=None, workspace=None,
+                     stream=None, expand=False):
+    """IKBO-LCB.  Returns ``(y_req [R,o_r,d], y_cand [C,o_c,d])``; see ``rocs_lcb_forward`` in the header.
+
+    ``expand=True`` runs the explicit-expand ablation (``rocs_lcb_forward_expand``) instead.
+    """
+    lib = load_library()
+    a, keep, y_req, y_cand = _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y_cand)
+    size_fn = lib.rocs_lcb_expand_workspace_size if expand else lib.rocs_lcb_workspace_size
+    nbytes = size_fn(ctypes.byref(a))
+    if nbytes == 0:
+        _check(lib.rocs_lcb_forward(ctypes.byref(a), _stream(stream)), "rocs_lcb_forward")  # reports the reason
+    ws = _workspace(nbytes, x_req.device, workspace)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    fn = lib.rocs_lcb_forward_expand if expand else lib.rocs_lcb_forward
+    _check(fn(ctypes.byref(a), _stream(stream)), fn.__name__)
+    rocs_lcb_forward.last_workspace = ws
+    return y_req, y_cand
+
+
+def rocs_lcb_forward_expand(*args, **kw):
+    return rocs_lcb_forward(*args, expand=True, **kw)
+
+
+def _dca_args(q_t, k_t, v_t, cand_off, seq_off, q_tokens, scale, o, lse):
+    dev = q_t.device
+    co_d, co_h = _offsets(cand_off, dev)
+    so_d, so_h = _offsets(seq_off, dev)
+    R = len(co_h) - 1
+    H, dh = k_t.shape[1], k_t.shape[2]
+    if o is None:
+        o = torch.empty(q_t.shape, dtype=torch.bfloat16, device=dev)
+    if lse is True:
+        lse = torch.empty(q_t.shape[:2], dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    for t in (q_t, k_t, v_t, o):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16):
+            raise RocsError(1, "DCA tensors must be contiguous bf16 CUDA tensors")
+    a = DcaArgs(R=R, q=q_tokens, H=H, dh=dh, scale=float(scale),
+                cand_off_dev=co_d.data_ptr(), cand_off_host=co_h.ctypes.data,
+                seq_off_dev=so_d.data_ptr(), seq_off_host=so_h.ctypes.data,
+                q_ptr=q_t.data_ptr() if q_t.numel() else None, k_ptr=k_t.data_ptr() if k_t.numel() else None,
+                v_ptr=v_t.data_ptr() if v_t.numel() else None, o_ptr=o.data_ptr() if o.numel() else None,
+                lse_ptr=lse.data_ptr() if lse is not None else None)
+    return a, (co_d, co_h, so_d, so_h), o, lse
+
+
+def rocs_dca_forward(q_t, k_t, v_t, cand_off, seq_off, q_tokens, scale, o=None, lse=True, workspace=None,
+                     stream=None, expand_chunk=None):
+    """IKBO-DCA.  Returns ``(o [C*q,H,dh], lse [C*q,H] or None)``.
+
+    ``expand_chunk=n`` runs the explicit-expand ablation with chunks of n candidates.
+    """
+    lib = load_library()
+    a, keep, o, lse = _dca_args(q_t, k_t, v_t, cand_off, seq_off, q_tokens, scale, o, lse)
+    if expand_chunk:
+        nbytes = lib.rocs_dca_expand_workspace_size(ctypes.byref(a), int(expand_chunk))
+    else:
+        nbytes = lib.rocs_dca_workspace_size(ctypes.byref(a))
+    if nbytes == 0:
+        _check(lib.rocs_dca_forward(ctypes.byref(a), _stream(stream)), "rocs_dca_forward")
+    ws = _workspace(nbytes, q_t.device, workspace)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    if expand_chunk:
+        _check(lib.rocs_dca_forward_expand(ctypes.byref(a), int(expand_chunk), _stream(stream)),
+               "rocs_dca_forward_expand")
+    else:
+        _check(lib.rocs_dca_forward(ctypes.byref(a), _stream(stream)), "rocs_dca_forward")
+    rocs_dca_forward.last_workspace = ws
+    return o, lse
+
+
+def rocs_dca_forward_expand(*args, expand_chunk=1024, **kw):
+    return rocs_dca_forward(*args, expand_chunk=expand_chunk, **kw)
+
+
+def rocs_proj_forward(inp, w, out=None, workspace=None, stream=None):
+    """``out[M, N] = inp[M, K] . w[N, K]^T`` (bf16)."""
+    lib = load_library()
+    M, K = inp.shape[0], int(np.prod(inp.shape[1:]))
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=inp.device)
+    for t in (inp, w, out):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16):
+            raise RocsError(1, "projection tensors must be contiguous bf16 CUDA tensors")
+    a = ProjArgs(M=M, N=N, K=K, in_=inp.data_ptr() if M else None, w=w.data_ptr(), out=out.data_ptr() if M else None)
+    ws = _workspace(lib.rocs_proj_workspace_size(ctypes.byref(a)), inp.device, workspace)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check(lib.rocs_proj_forward(ctypes.byref(a), _stream(stream)), "rocs_proj_forward")
+    rocs_proj_forward.last_workspace = ws
+    return out
+
+
+def rocs_read_status(workspace, stream=None):
+    """Synchronise the stream and return ``(device_code, detail)`` of a workspace."""
+    lib = load_library()
+    code, detail = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib.rocs_read_status(_ptr(workspace), _stream(stream), ctypes.byref(code), ctypes.byref(detail)),
+           "rocs_read_status")
+    return code.value, detail.value
+
+
+def chain_forward(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, w_q, k_t, v_t, seq_off, heads, head_dim, scale,
+                  stream=None, workspaces=None):
+    """Chained block: IKBO-LCB -> query projection -> IKBO-DCA (one query token per candidate).
+
+    Returns ``(y_req, y_cand, q, o, lse)``.  Three C-ABI calls on one stream; intermediates stay bf16 in HBM.
+    """
+    ws = workspaces or {}
+    y_req, y_cand = rocs_lcb_forward(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, workspace=ws.get("lcb"),
+                                     stream=stream)
+    C = y_cand.shape[0]
+    q = rocs_proj_forward(y_cand.view(C, -1), w_q, workspace=ws.get("proj"), stream=stream)
+    o, lse = rocs_dca_forward(q.view(C, heads, head_dim), k_t, v_t, cand_off, seq_off, 1, scale,
+                              workspace=ws.get("dca"), stream=stream)
+    return y_req, y_cand, q, o, lse

@@ -1,0 +1,517 @@
+// dca_sm100.cu -- IKBO-DCA on B200: persistent flash-style cross attention over K/V that is
+// stored once per request.
+//
+// Computes the candidate-group cross attention of "ROCS: Request-Oriented Compute Sharing ..."
+// (arXiv:2607.27744; paper-archivist notes, section 3.2, Eq. (13)),
+//     O_i = softmax(scale . Q_i K_{m_i}^T) V_{m_i}        (non-causal),
+// resolving m_i inside the kernel (section 4.3.1): K/V stay at batch size B_r and every
+// candidate of a request reads the same physical K/V tiles.
+//
+// sm_100a design (the pages' design targeted Hopper warp-group MMA; what carries over is
+// "stack many short candidate queries of one request into a full query tile" and
+// "persistent, warp-specialised, pipelined across tiles"):
+//   * work unit = (request r, head h, 256 consecutive query rows of r).  The query rows of
+//     ALL candidates of r are one M dimension (q tokens per candidate, candidates
+//     contiguous), so two 128-row tcgen05 tiles (A and B) are filled with many candidates
+//     and share every K/V tile loaded into shared memory (section 4.3.2's "several
+//     candidates per CTA", generalised).  Tiles never cross requests.
+//   * warp roles: warp 0 TMA producer (Q tiles, then K/V tiles in consumption order through
+//     one ring), warp 1 single-thread tcgen05.mma issuer, warps 4-7 softmax/epilogue of
+//     tile A, warps 8-11 of tile B.  S = Q K^T lands in TMEM (fp32), the softmax warps write
+//     P (bf16) back over S in TMEM, and P V is issued with P as the TMEM A operand, O
+//     accumulating in TMEM.  The issuer alternates [PV_A, S_A] and [PV_B, S_B] so the
+//     tensor core works on one tile while the softmax warps of the other tile run.
+//   * online softmax in the exp2 domain with lazy rescaling: O and the running sum are
+//     rescaled only when a row's maximum grows by more than 2^8.
+//   * work units are claimed from a global ticket in a table ordered longest request first
+//     (load balance), units of one (request, head) adjacent (K/V L2 locality; section 4.3.1's
+//     grid reordering, expressed as the claim order of a persistent kernel).
+#include "lcb_sm100.h"
+
+namespace rocs {
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kSoftmaxWarp0 = 4;  // warps 4..7 tile A, 8..11 tile B
+constexpr int BM = 128, BN = 128;
+constexpr int kRowsPerUnit = 2 * BM;
+
+template <int DH>
+struct DcaSmem {
+  static constexpr uint32_t kTile = BM * DH * 2;  // one Q tile or one K/V tile (bf16)
+  static constexpr int kRing = DH == 128 ? 5 : 10;
+  static constexpr uint32_t off_q = 0;
+  static constexpr uint32_t off_ring = 2 * kTile;
+  static constexpr uint32_t off_bar = off_ring + kRing * kTile;
+  static constexpr uint32_t n_bars = 2 * kRing + 2 * 8 + 1;
+  static constexpr uint32_t off_misc = off_bar + n_bars * 8;
+  static constexpr uint32_t bytes = off_misc + 64;
+  static constexpr uint32_t alloc_bytes = bytes + 1024;
+  static_assert(alloc_bytes <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+struct Unit {
+  int r, h, row0;  // request, head, first query row (within the request's rows)
+  int rows;        // query rows of the request (q * N_r)
+  int qbase;       // global query row of the request's first row (q * cand_off[r])
+  int s0, L;       // first key row, number of keys
+  int nkv;         // K/V tiles
+  bool hasB;       // second 128-row tile has at least one valid row
+};
+
+__device__ __forceinline__ Unit load_unit(const DcaParams& p, int u) {
+  const int4 e = p.units[u];
+  Unit w;
+  w.r = e.x;
+  w.h = e.y;
+  w.row0 = e.z;
+  const int c0 = p.cand_off[w.r], c1 = p.cand_off[w.r + 1];
+  w.rows = p.q * (c1 - c0);
+  w.qbase = p.q * c0;
+  w.s0 = p.seq_off[w.r];
+  w.L = p.seq_off[w.r + 1] - w.s0;
+  w.nkv = (w.L + BN - 1) / BN;
+  w.hasB = w.row0 + BM < w.rows;
+  return w;
+}
+
+}  // namespace
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __grid_constant__ DcaParams p) {
+  using L = DcaSmem<DH>;
+  constexpr int kRing = L::kRing;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_q = smem + L::off_q;
+  uint8_t* s_ring = smem + L::off_ring;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
+  uint64_t* ring_full = bars;
+  uint64_t* ring_empty = bars + kRing;
+  uint64_t* q_full = bars + 2 * kRing;  // [2]
+  uint64_t* q_empty = q_full + 2;
+  uint64_t* s_full = q_empty + 2;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* o_empty = o_full + 2;
+  uint64_t* wq_full = o_empty + 2;  // two-slot work queue: the producer runs one unit ahead
+  uint64_t* wq_empty = wq_full + 2;
+  uint64_t* drain_bar = wq_empty + 2;
+  int* s_wq = reinterpret_cast<int*>(smem + L::off_misc);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::off_misc + 16);
+  int* s_abort = reinterpret_cast<int*>(smem + L::off_misc + 32);
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = threadIdx.x & 31;
+  const Ctl ctl{s_abort, p.ws};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&ring_full[s], 1);
+      mbar_init(&ring_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 4);
+      mbar_init(&o_full[x], 1);
+      mbar_init(&o_empty[x], 4);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&wq_full[k], 1);
+      mbar_init(&wq_empty[k], 1 + 8);
+    }
+    mbar_init(drain_bar, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+DH) O_B [256+DH,256+2DH); P_X over S_X [0,64)
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      uint32_t rs = 0, rph = 0, ws_ = 0, wph = 0, qeph[2] = {0, 0};
+      int n_issued = 0;
+      bool ok = true;
+      auto load_kv = [&](const CUtensorMap* tm, int y, int x0) -> bool {
+        if (!mbar_wait(&ring_empty[rs], rph ^ 1, ctl, 501)) return false;
+        uint8_t* slot = s_ring + rs * L::kTile;
+        mbar_arrive_expect_tx(&ring_full[rs], L::kTile);
+#pragma unroll
+        for (int cc = 0; cc < DH / 64; ++cc) tma_load_2d(slot + cc * (BM * 128), tm, &ring_full[rs], x0 + cc * 64, y);
+        ++n_issued;
+        if (++rs == kRing) { rs = 0; rph ^= 1; }
+        return true;
+      };
+      while (ok) {
+        const int t = atomicAdd(&p.ws->counter, 1);
+        const int item = t < p.n_units ? t : -1;
+        if (!mbar_wait(&wq_empty[ws_], wph ^ 1, ctl, 502)) { ok = false; break; }
+        s_wq[ws_] = item;
+        mbar_arrive(&wq_full[ws_]);
+        if (++ws_ == 2) { ws_ = 0; wph ^= 1; }
+        if (item < 0) break;
+        const Unit w = load_unit(p, item);
+        if (w.nkv == 0) continue;
+        const int x0 = w.h * DH;
+        for (int x = 0; x < (w.hasB ? 2 : 1); ++x) {
+          if (!mbar_wait(&q_empty[x], qeph[x] ^ 1, ctl, 503)) { ok = false; break; }
+          qeph[x] ^= 1;
+          mbar_arrive_expect_tx(&q_full[x], L::kTile);
+#pragma unroll
+          for (int cc = 0; cc < DH / 64; ++cc)
+            tma_load_2d(s_q + x * L::kTile + cc * (BM * 128), &p.tm_q, &q_full[x], x0 + cc * 64,
+                        w.qbase + w.row0 + x * BM);
+        }
+        if (!ok) break;
+        // K/V in the order the MMA issuer consumes them: K0, (K1, V0), (K2, V1), ..., V_last
+        ok = load_kv(&p.tm_k, w.s0, x0);
+        for (int j = 1; ok && j < w.nkv; ++j) {
+          ok = load_kv(&p.tm_k, w.s0 + j * BN, x0);
+          if (ok) ok = load_kv(&p.tm_v, w.s0 + (j - 1) * BN, x0);
+        }
+        if (ok) ok = load_kv(&p.tm_v, w.s0 + (w.nkv - 1) * BN, x0);
+      }
+      if (!ok) {
+        for (int k = n_issued > kRing ? n_issued - kRing : 0; k < n_issued; ++k)
+          mbar_drain(&ring_full[k % kRing], (k / kRing) & 1, 20000000ull);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ tcgen05 issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);  // S = Q K^T : both K-major
+      constexpr uint32_t idesc_o = idesc_bf16(BM, DH, false, true);   // O += P V  : V is MN-major
+      uint32_t rs = 0, rph = 0, ws_ = 0, wph = 0;
+      uint32_t qfph[2] = {0, 0}, pph[2] = {0, 0}, oeph[2] = {0, 0};
+      bool ok = true;
+      const uint32_t q0 = smem_u32(s_q);
+      auto next_slot = [&](uint32_t& slot_addr, int where) -> bool {
+        if (!mbar_wait(&ring_full[rs], rph, ctl, where)) return false;
+        slot_addr = smem_u32(s_ring + rs * L::kTile);
+        return true;
+      };
+      auto release_slot = [&](uint32_t slot_addr) {  // slots are consumed in ring order
+        const uint32_t idx = (slot_addr - smem_u32(s_ring)) / L::kTile;
+        umma_commit(&ring_empty[idx]);
+      };
+      auto advance = [&]() {
+        if (++rs == kRing) { rs = 0; rph ^= 1; }
+      };
+      auto issue_s = [&](int x, uint32_t kslot) {
+        const uint32_t qa = q0 + x * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk)
+          umma_ss(tmem_base + x * 128, sdesc_sw128(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(kslot + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024), idesc_s, kk != 0);
+        umma_commit(&s_full[x]);
+      };
+      auto issue_pv = [&](int x, uint32_t vslot, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts(tmem_base + 256 + x * DH, tmem_base + x * 128 + kk * 8,
+                  sdesc_sw128(vslot + kk * 2048, BN * 128, 1024), idesc_o, (acc || kk != 0) ? 1u : 0u);
+      };
+      auto wait_p = [&](int x, bool first_pv) -> bool {
+        if (!mbar_wait(&p_full[x], pph[x], ctl, 601)) return false;
+        pph[x] ^= 1;
+        if (first_pv) {  // O_x of the previous unit must have been read out
+          if (!mbar_wait(&o_empty[x], oeph[x] ^ 1, ctl, 602)) return false;
+          oeph[x] ^= 1;
+        }
+        tc_fence_after();
+        return true;
+      };
+      for (;;) {
+        if (!mbar_wait(&wq_full[ws_], wph, ctl, 603)) { ok = false; break; }
+        const int item = s_wq[ws_];
+        mbar_arrive(&wq_empty[ws_]);
+        if (++ws_ == 2) { ws_ = 0; wph ^= 1; }
+        if (item < 0) break;
+        const Unit w = load_unit(p, item);
+        if (w.nkv == 0) continue;
+        const int nx = w.hasB ? 2 : 1;
+        for (int x = 0; x < nx && ok; ++x) {
+          if (!mbar_wait(&q_full[x], qfph[x], ctl, 604)) ok = false;
+          qfph[x] ^= 1;
+        }
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t kslot, vslot;
+        if (!next_slot(kslot, 605)) { ok = false; break; }
+        advance();
+        tc_fence_after();
+        issue_s(0, kslot);
+        if (nx == 2) issue_s(1, kslot);
+        release_slot(kslot);
+        for (int j = 1; j < w.nkv; ++j) {
+          if (!next_slot(kslot, 606)) { ok = false; break; }
+          advance();
+          if (!next_slot(vslot, 607)) { ok = false; break; }
+          advance();
+          for (int x = 0; x < nx; ++x) {
+            if (!wait_p(x, j == 1)) { ok = false; break; }
+            issue_pv(x, vslot, j > 1);
+            issue_s(x, kslot);
+          }
+          if (!ok) break;
+          release_slot(vslot);
+          release_slot(kslot);
+        }
+        if (!ok) break;
+        for (int x = 0; x < nx; ++x) umma_commit(&q_empty[x]);
+        if (!next_slot(vslot, 608)) { ok = false; break; }
+        advance();
+        for (int x = 0; x < nx; ++x) {
+          if (!wait_p(x, w.nkv == 1)) { ok = false; break; }
+          issue_pv(x, vslot, w.nkv > 1);
+          umma_commit(&o_full[x]);
+        }
+        if (!ok) break;
+        release_slot(vslot);
+      }
+      umma_commit(drain_bar);
+      mbar_drain(drain_bar, 0, 50000000ull);
+    }
+  } else if (warp >= kSoftmaxWarp0) {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int x = (warp - kSoftmaxWarp0) >> 2;  // 0: tile A, 1: tile B
+    const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
+    const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
+    const uint32_t s_addr = tmem_base + t_lane + x * 128;
+    const uint32_t o_addr = tmem_base + t_lane + 256 + x * DH;
+    const float c = p.scale_log2;
+    uint32_t ws_ = 0, wph = 0, sph = 0, ofph = 0;
+    bool ok = true;
+    for (;;) {
+      if (!mbar_wait(&wq_full[ws_], wph, ctl, 701)) { ok = false; break; }
+      const int item = s_wq[ws_];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wq_empty[ws_]);
+      if (++ws_ == 2) { ws_ = 0; wph ^= 1; }
+      if (item < 0) break;
+      const Unit w = load_unit(p, item);
+      if (x == 1 && !w.hasB) continue;
+      const int row = w.row0 + x * BM + 32 * quarter + (int)lane;  // row within the request
+      const bool row_ok = row < w.rows;
+      __nv_bfloat16* orow = p.o + ((size_t)(w.qbase + row) * p.H + w.h) * DH;
+      if (w.nkv == 0) {  // request without keys: O = 0, LSE = -inf
+        if (row_ok) {
+#pragma unroll
+          for (int k = 0; k < DH / 8; ++k) st_global_v4(orow + 8 * k, 0u, 0u, 0u, 0u);
+          if (p.lse) p.lse[(size_t)(w.qbase + row) * p.H + w.h] = -INFINITY;
+        }
+        continue;
+      }
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < w.nkv; ++j) {
+        if (!mbar_wait(&s_full[x], sph, ctl, 702)) { ok = false; break; }
+        sph ^= 1;
+        tc_fence_after();
+        uint32_t sv[4][32];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + c4 * 32, sv[c4]);
+        tmem_ld_wait();
+        const int kvalid = w.L - j * BN;
+        if (kvalid < BN) {
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (c4 * 32 + k >= kvalid) sv[c4][k] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(sv[c4][k]));
+        const float mxs = mx * c;
+        if (j == 0) {
+          m_used = mxs;
+        } else if (__any_sync(0xffffffffu, mxs > m_used + 8.0f)) {
+          const float m_new = fmaxf(m_used, mxs);
+          const float f = ex2(m_used - m_new);
+          l *= f;
+#pragma unroll 1
+          for (int cc = 0; cc < DH / 32; ++cc) {
+            uint32_t ov[32];
+            tmem_ld32(o_addr + cc * 32, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+            tmem_st32(o_addr + cc * 32, ov);
+          }
+          m_used = m_new;
+        }
+        const float nm = -m_used;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float p0 = ex2(fmaf(__uint_as_float(sv[c4][2 * k]), c, nm));
+            const float p1 = ex2(fmaf(__uint_as_float(sv[c4][2 * k + 1]), c, nm));
+            lsum += p0 + p1;
+            pk[k] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(s_addr + c4 * 16, pk);  // P (bf16 pairs) over the first 64 columns of S
+        }
+        l += lsum;
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[x]);
+      }
+      if (!ok) break;
+      if (!mbar_wait(&o_full[x], ofph, ctl, 703)) { ok = false; break; }
+      ofph ^= 1;
+      tc_fence_after();
+      const float inv = 1.0f / l;
+#pragma unroll 1
+      for (int cc = 0; cc < DH / 32; ++cc) {
+        uint32_t ov[32];
+        tmem_ld32(o_addr + cc * 32, ov);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            st_global_v4(orow + cc * 32 + 8 * k,
+                         pack_bf16x2(__uint_as_float(ov[8 * k + 0]) * inv, __uint_as_float(ov[8 * k + 1]) * inv),
+                         pack_bf16x2(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv),
+                         pack_bf16x2(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv),
+                         pack_bf16x2(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[x]);
+      if (row_ok && p.lse) p.lse[(size_t)(w.qbase + row) * p.H + w.h] = (m_used + lg2(l)) * 0.69314718055994531f;
+    }
+    (void)ok;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// Work-unit table: one block.  units_r = H * ceil(q*N_r / 256); requests ordered by key
+// length descending (ties by index) so the longest units are claimed first.
+// Scratch (workspace): len[R], sorted[R], start[R+1].
+// ------------------------------------------------------------------------------------
+__global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
+  int* len = p.scratch;
+  int* sorted = len + p.R;
+  int* start = sorted + p.R;
+  __shared__ int s_part[1024];
+  const int R = p.R, T = blockDim.x, t = threadIdx.x;
+  for (int r = t; r < R; r += T) len[r] = p.seq_off[r + 1] - p.seq_off[r];
+  __syncthreads();
+  // rank by (len desc, index asc); identity order for very many requests
+  for (int r = t; r < R; r += T) {
+    int rank = r;
+    if (R <= 8192) {
+      rank = 0;
+      const int lr = len[r];
+      for (int k = 0; k < R; ++k) {
+        const int lk = len[k];
+        rank += (lk > lr) || (lk == lr && k < r);
+      }
+    }
+    sorted[rank] = r;
+  }
+  __syncthreads();
+  // units of each sorted position, exclusive scan over positions
+  const int per = (R + T - 1) / T;
+  const int b0 = min(R, t * per), b1 = min(R, b0 + per);
+  int sum = 0;
+  for (int k = b0; k < b1; ++k) {
+    const int r = sorted[k];
+    const int rows = p.q * (p.cand_off[r + 1] - p.cand_off[r]);
+    sum += p.H * ((rows + p.rows_per_unit - 1) / p.rows_per_unit);
+  }
+  s_part[t] = sum;
+  __syncthreads();
+  for (int off = 1; off < T; off <<= 1) {
+    const int v = t >= off ? s_part[t - off] : 0;
+    __syncthreads();
+    s_part[t] += v;
+    __syncthreads();
+  }
+  int run = s_part[t] - sum;
+  for (int k = b0; k < b1; ++k) {
+    const int r = sorted[k];
+    const int rows = p.q * (p.cand_off[r + 1] - p.cand_off[r]);
+    const int nb = (rows + p.rows_per_unit - 1) / p.rows_per_unit;
+    start[k] = run;
+    for (int h = 0; h < p.H; ++h)
+      for (int mb = 0; mb < nb; ++mb) {
+        const int u = run + h * nb + mb;
+        if (u < p.max_units) p.units[u] = make_int4(r, h, mb * p.rows_per_unit, 0);
+        else record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 801);
+      }
+    run += p.H * nb;
+  }
+  if (t == T - 1 && s_part[T - 1] != p.max_units) record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 802);
+  if (t == 0) p.ws->counter = 0;
+}
+
+cudaError_t launch_dca_schedule(const DcaSchedParams& p, cudaStream_t st) {
+  rocs_dca_schedule_kernel<<<1, 1024, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int DH>
+static cudaError_t launch_t(const DcaParams& p, int grid, cudaStream_t st) {
+  using L = DcaSmem<DH>;
+  auto k = rocs_dca_sm100_kernel<DH>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::alloc_bytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  k<<<grid, kThreads, L::alloc_bytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dca_sm100(const DcaParams& p, int dh, int grid, cudaStream_t st) {
+  if (dh == 128) return launch_t<128>(p, grid, st);
+  if (dh == 64) return launch_t<64>(p, grid, st);
+  return cudaErrorInvalidValue;
+}
+
+int dca_rows_per_unit() { return kRowsPerUnit; }
+
+}  // namespace rocs

@@ -1,0 +1,77 @@
+// lcb_sm100.h -- launch parameters of the IKBO kernels (internal to the library).
+#pragma once
+#include "sm100.cuh"
+
+namespace rocs {
+
+// Persistent IKBO-LCB kernel (bf16 in, fp32 accumulate, bf16 out).
+struct LcbParams {
+  CUtensorMap tm_xc;   // X^C  viewed as [C*n_c, d],  box {64, n_c}
+  CUtensorMap tm_xr;   // X^R  viewed as [R*n_r, d],  box {64, 64}
+  CUtensorMap tm_wcc;  // W_CC [o_c, n_c],            box {64, 128}
+  CUtensorMap tm_wrr;  // W_RR [o_r, n_r],            box {64, 128}
+  CUtensorMap tm_wcr;  // W_CR [o_c, n_r],            box {64, 128}
+  CUtensorMap tm_yc;   // Y^C  viewed as [C*o_c, d],  box {64, 32}  (stores)
+  CUtensorMap tm_yr;   // Y^R  viewed as [R*o_r, d],  box {64, 32}  (stores)
+  const int32_t* cand_off;  // [R+1]
+  float* zws;               // Z fp32, [R][d/4][o_c][4]
+  int* flags;               // [R], incremented by each epilogue warp of the Z tile
+  WsHeader* ws;
+  int R, C, n_r, o_r;
+};
+cudaError_t launch_lcb_sm100(const LcbParams& p, int d, int n_c, int grid, cudaStream_t st);
+
+// fp32 CUDA-core IKBO-LCB (two launches: request GEMM, then candidate GEMM + fused Z add).
+struct LcbF32Params {
+  const float *x_req, *x_cand, *w_rr, *w_cr, *w_cc;
+  float *y_req, *y_cand, *z;  // z: [R, o_c, d]
+  const int32_t* cand_off;
+  WsHeader* ws;
+  int R, C, n_r, n_c, d, o_r, o_c;
+};
+cudaError_t launch_lcb_f32(const LcbF32Params& p, cudaStream_t st);
+
+// Persistent IKBO-DCA kernel.
+struct DcaParams {
+  CUtensorMap tm_q;  // Q viewed as [C*q, H*dh], box {64, 128}
+  CUtensorMap tm_k;  // K viewed as [T, H*dh],   box {64, 128}
+  CUtensorMap tm_v;  // V viewed as [T, H*dh],   box {64, 128}
+  const int32_t* cand_off;
+  const int32_t* seq_off;
+  const int4* units;  // work-unit table {r, h, row0, 0}
+  __nv_bfloat16* o;
+  float* lse;
+  WsHeader* ws;
+  int R, q, H, n_units;
+  float scale_log2;  // softmax scale * log2(e)
+};
+cudaError_t launch_dca_sm100(const DcaParams& p, int dh, int grid, cudaStream_t st);
+
+struct DcaSchedParams {
+  const int32_t* cand_off;
+  const int32_t* seq_off;
+  int* scratch;  // 3R+1 ints
+  int4* units;
+  WsHeader* ws;
+  int R, q, H, rows_per_unit, max_units;
+};
+cudaError_t launch_dca_schedule(const DcaSchedParams& p, cudaStream_t st);
+
+// Dense projection GEMM  out[M, N] = in[M, K] . W[N, K]^T  (bf16 in/out, fp32 accumulate).
+struct ProjParams {
+  CUtensorMap tm_a;    // in  [M, K], box {64, 128}
+  CUtensorMap tm_b;    // W   [N, K], box {64, 256}
+  __nv_bfloat16* out;  // [M, N]
+  WsHeader* ws;
+  int M, N, K;
+};
+cudaError_t launch_proj_sm100(const ProjParams& p, int grid, cudaStream_t st);
+
+// Explicit-expand baseline helpers.
+cudaError_t launch_expand_rows(const void* src, void* dst, const int32_t* cand_off, int R, int C, int64_t row_bytes,
+                               int64_t rows_per_item, cudaStream_t st);
+cudaError_t launch_expand_kv(const void* k, const void* v, void* k_out, void* v_out, const int32_t* cand_off,
+                             const int32_t* seq_off, int32_t* seq_off_out, int R, int c0, int c1, int64_t row_bytes,
+                             cudaStream_t st);
+
+}  // namespace rocs

@@ -1,0 +1,390 @@
+// rocs_abi.cu -- host side of the C ABI declared in include/rocs_ikbo.h: argument and CSR
+// validation, workspace layout, TMA tensor-map construction and kernel launches.
+// No entry point allocates or frees memory or synchronises a stream (except
+// rocs_read_status, whose job is to synchronise and read).
+#include <cstring>
+
+#include "lcb_sm100.h"
+
+namespace rocs {
+int dca_rows_per_unit();
+}
+
+using namespace rocs;
+
+namespace {
+
+thread_local int g_last_launches = 0;
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return n;
+  static int cache[64] = {0};
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map [outer rows, inner cols] with a row pitch, 128-byte swizzle.
+bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_in,
+               uint32_t box_out) {
+  EncodeTiledFn f = encode_fn();
+  if (!f || !base || inner == 0 || outer == 0) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_in, box_out};
+  cuuint32_t es[2] = {1, 1};
+  return f(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// off[0] == 0, non-decreasing; *total = off[R]
+int check_csr(const int32_t* off, int64_t R, int64_t* total) {
+  if (!off) return ROCS_ERR_INVALID_ARG;
+  if (off[0] != 0) return ROCS_ERR_BAD_OFFSETS;
+  for (int64_t r = 0; r < R; ++r)
+    if (off[r + 1] < off[r]) return ROCS_ERR_BAD_OFFSETS;
+  *total = off[R];
+  return ROCS_OK;
+}
+
+// ---------------------------------------------------------------- LCB
+// workspace = [WsHeader][body]; body = [flags: R ints][Z: R * o_c * d fp32]
+struct LcbLayout {
+  size_t flags, z, body;
+};
+LcbLayout lcb_body(int64_t R, int64_t o_c, int64_t d) {
+  LcbLayout L;
+  L.flags = 0;
+  L.z = a256((size_t)R * sizeof(int));
+  L.body = L.z + (size_t)R * o_c * d * sizeof(float);
+  return L;
+}
+size_t lcb_bytes(const rocs_lcb_args* a) { return sizeof(WsHeader) + lcb_body(a->R, a->o_c, a->d).body; }
+
+int lcb_validate(const rocs_lcb_args* a, int64_t* C) {
+  if (!a) return ROCS_ERR_INVALID_ARG;
+  if (a->R < 0 || a->n_r <= 0 || a->n_c <= 0 || a->d <= 0 || a->o_r <= 0 || a->o_c <= 0) return ROCS_ERR_INVALID_ARG;
+  if (a->R > (1 << 30)) return ROCS_ERR_UNSUPPORTED;
+  if (a->dtype != ROCS_F32 && a->dtype != ROCS_BF16) return ROCS_ERR_INVALID_ARG;
+  int rc = check_csr(a->cand_off_host, a->R, C);
+  if (rc) return rc;
+  if (a->R > 0 && !a->cand_off_dev) return ROCS_ERR_INVALID_ARG;
+  const int64_t es = a->dtype == ROCS_BF16 ? 2 : 4;
+  if ((a->d * es) % 16 != 0) return ROCS_ERR_UNSUPPORTED;  // row alignment contract
+  if (a->R > 0 && (!a->x_req || !a->w_rr || !a->w_cr || !a->w_cc || !a->y_req)) return ROCS_ERR_INVALID_ARG;
+  if (*C > 0 && (!a->x_cand || !a->y_cand)) return ROCS_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->x_req, a->x_cand, a->w_rr, a->w_cr, a->w_cc, a->y_req, a->y_cand};
+  for (const void* p : ptrs)
+    if (p && !al16(p)) return ROCS_ERR_INVALID_ARG;
+  if (a->dtype == ROCS_BF16) {
+    if (a->n_r % 64 || (a->n_c != 64 && a->n_c != 128) || (a->d != 64 && a->d != 128) || a->o_r % 128 ||
+        a->o_c != 128)
+      return ROCS_ERR_UNSUPPORTED;
+    if ((a->n_r * 2) % 16 || (a->n_c * 2) % 16) return ROCS_ERR_UNSUPPORTED;
+    if (*C * a->o_c >= (int64_t(1) << 31) || a->R * a->n_r >= (int64_t(1) << 31) || *C * a->n_c >= (int64_t(1) << 31))
+      return ROCS_ERR_UNSUPPORTED;  // TMA coordinates are 32-bit
+  } else {
+    if (a->n_r > 1024 || a->n_c > 1024 || a->d > 1024) return ROCS_ERR_UNSUPPORTED;
+  }
+  return ROCS_OK;
+}
+
+int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaStream_t st, int* launches) {
+  const LcbLayout L = lcb_body(a->R, a->o_c, a->d);
+  if (w == reinterpret_cast<uint8_t*>(hdr + 1)) {
+    if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader) + (size_t)a->R * sizeof(int), st) != cudaSuccess) return ROCS_ERR_CUDA;
+  } else if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess ||
+             cudaMemsetAsync(w, 0, (size_t)a->R * sizeof(int), st) != cudaSuccess) {
+    return ROCS_ERR_CUDA;
+  }
+  if (a->R == 0) return ROCS_OK;
+  if (a->dtype == ROCS_F32) {
+    LcbF32Params p;
+    p.x_req = static_cast<const float*>(a->x_req);
+    p.x_cand = static_cast<const float*>(a->x_cand);
+    p.w_rr = static_cast<const float*>(a->w_rr);
+    p.w_cr = static_cast<const float*>(a->w_cr);
+    p.w_cc = static_cast<const float*>(a->w_cc);
+    p.y_req = static_cast<float*>(a->y_req);
+    p.y_cand = static_cast<float*>(a->y_cand);
+    p.z = reinterpret_cast<float*>(w + L.z);
+    p.cand_off = a->cand_off_dev;
+    p.ws = hdr;
+    p.R = (int)a->R;
+    p.C = (int)C;
+    p.n_r = (int)a->n_r;
+    p.n_c = (int)a->n_c;
+    p.d = (int)a->d;
+    p.o_r = (int)a->o_r;
+    p.o_c = (int)a->o_c;
+    if (launch_lcb_f32(p, st) != cudaSuccess) return ROCS_ERR_CUDA;
+    *launches = C > 0 ? 2 : 1;
+    return ROCS_OK;
+  }
+  LcbParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint64_t d = a->d, rb = d * 2;
+  bool ok = true;
+  if (C > 0) {
+    ok &= tmap_bf16(&p.tm_xc, a->x_cand, d, (uint64_t)C * a->n_c, rb, 64, (uint32_t)a->n_c);
+    ok &= tmap_bf16(&p.tm_yc, a->y_cand, d, (uint64_t)C * a->o_c, rb, 64, 32);
+    ok &= tmap_bf16(&p.tm_wcc, a->w_cc, a->n_c, a->o_c, a->n_c * 2, 64, 128);
+  }
+  ok &= tmap_bf16(&p.tm_xr, a->x_req, d, (uint64_t)a->R * a->n_r, rb, 64, 64);
+  ok &= tmap_bf16(&p.tm_wrr, a->w_rr, a->n_r, a->o_r, a->n_r * 2, 64, 128);
+  ok &= tmap_bf16(&p.tm_wcr, a->w_cr, a->n_r, a->o_c, a->n_r * 2, 64, 128);
+  ok &= tmap_bf16(&p.tm_yr, a->y_req, d, (uint64_t)a->R * a->o_r, rb, 64, 32);
+  if (!ok) return ROCS_ERR_CUDA;
+  p.cand_off = a->cand_off_dev;
+  p.zws = reinterpret_cast<float*>(w + L.z);
+  p.flags = reinterpret_cast<int*>(w + L.flags);
+  p.ws = hdr;
+  p.R = (int)a->R;
+  p.C = (int)C;
+  p.n_r = (int)a->n_r;
+  p.o_r = (int)a->o_r;
+  const int64_t n_req_tiles = a->R * (1 + a->o_r / 128);
+  int64_t grid = C > n_req_tiles ? C : n_req_tiles;
+  if (grid > sm_count()) grid = sm_count();
+  if (grid < 1) grid = 1;
+  if (launch_lcb_sm100(p, (int)a->d, (int)a->n_c, (int)grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  *launches = 1;
+  return ROCS_OK;
+}
+
+// ---------------------------------------------------------------- DCA
+// workspace = [WsHeader][body]; body = [scratch: 3R+1 ints][work units: n_units int4]
+int64_t dca_units(const rocs_dca_args* a) {
+  const int rpu = dca_rows_per_unit();
+  int64_t n = 0;
+  for (int64_t r = 0; r < a->R; ++r) {
+    const int64_t rows = a->q * (int64_t)(a->cand_off_host[r + 1] - a->cand_off_host[r]);
+    n += a->H * ((rows + rpu - 1) / rpu);
+  }
+  return n;
+}
+struct DcaLayout {
+  size_t scratch, units, body;
+};
+DcaLayout dca_body(int64_t R, int64_t n_units) {
+  DcaLayout L;
+  L.scratch = 0;
+  L.units = a256((size_t)(3 * R + 1) * sizeof(int));
+  L.body = L.units + (size_t)n_units * sizeof(int4);
+  return L;
+}
+
+int dca_validate(const rocs_dca_args* a, int64_t* C, int64_t* T) {
+  if (!a) return ROCS_ERR_INVALID_ARG;
+  if (a->R < 0 || a->q <= 0 || a->H <= 0 || a->dh <= 0) return ROCS_ERR_INVALID_ARG;
+  if (a->dh != 64 && a->dh != 128) return ROCS_ERR_UNSUPPORTED;
+  if (a->R > (1 << 28)) return ROCS_ERR_UNSUPPORTED;
+  int rc = check_csr(a->cand_off_host, a->R, C);
+  if (rc) return rc;
+  rc = check_csr(a->seq_off_host, a->R, T);
+  if (rc) return rc;
+  if (a->R > 0 && (!a->cand_off_dev || !a->seq_off_dev)) return ROCS_ERR_INVALID_ARG;
+  if (*C > 0 && (!a->q_ptr || !a->o_ptr)) return ROCS_ERR_INVALID_ARG;
+  if (*T > 0 && (!a->k_ptr || !a->v_ptr)) return ROCS_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->q_ptr, a->k_ptr, a->v_ptr, a->o_ptr};
+  for (const void* p : ptrs)
+    if (p && !al16(p)) return ROCS_ERR_INVALID_ARG;
+  if (a->lse_ptr && (reinterpret_cast<uintptr_t>(a->lse_ptr) & 3u)) return ROCS_ERR_INVALID_ARG;
+  if (*C * a->q >= (int64_t(1) << 31) || *T >= (int64_t(1) << 31) || a->H * a->dh >= (int64_t(1) << 20))
+    return ROCS_ERR_UNSUPPORTED;
+  return ROCS_OK;
+}
+
+int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHeader* hdr, uint8_t* w,
+            cudaStream_t st, int* launches) {
+  const DcaLayout L = dca_body(a->R, n_units);
+  if (n_units >= (int64_t(1) << 31)) return ROCS_ERR_UNSUPPORTED;
+  if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return ROCS_ERR_CUDA;
+  if (n_units == 0) return ROCS_OK;
+  DcaSchedParams sp;
+  sp.cand_off = a->cand_off_dev;
+  sp.seq_off = a->seq_off_dev;
+  sp.scratch = reinterpret_cast<int*>(w + L.scratch);
+  sp.units = reinterpret_cast<int4*>(w + L.units);
+  sp.ws = hdr;
+  sp.R = (int)a->R;
+  sp.q = (int)a->q;
+  sp.H = (int)a->H;
+  sp.rows_per_unit = dca_rows_per_unit();
+  sp.max_units = (int)n_units;
+  if (launch_dca_schedule(sp, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  DcaParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint64_t hd = a->H * a->dh, rb = hd * 2;
+  bool ok = tmap_bf16(&p.tm_q, a->q_ptr, hd, (uint64_t)C * a->q, rb, 64, 128);
+  if (T > 0) {
+    ok &= tmap_bf16(&p.tm_k, a->k_ptr, hd, (uint64_t)T, rb, 64, 128);
+    ok &= tmap_bf16(&p.tm_v, a->v_ptr, hd, (uint64_t)T, rb, 64, 128);
+  } else {  // never loaded (every request has zero keys); any valid descriptor will do
+    p.tm_k = p.tm_q;
+    p.tm_v = p.tm_q;
+  }
+  if (!ok) return ROCS_ERR_CUDA;
+  p.cand_off = a->cand_off_dev;
+  p.seq_off = a->seq_off_dev;
+  p.units = sp.units;
+  p.o = static_cast<__nv_bfloat16*>(a->o_ptr);
+  p.lse = a->lse_ptr;
+  p.ws = sp.ws;
+  p.R = (int)a->R;
+  p.q = (int)a->q;
+  p.H = (int)a->H;
+  p.n_units = (int)n_units;
+  p.scale_log2 = a->scale * 1.4426950408889634f;
+  int64_t grid = n_units < sm_count() ? n_units : sm_count();
+  if (launch_dca_sm100(p, (int)a->dh, (int)grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  *launches = 2;
+  return ROCS_OK;
+}
+
+}  // namespace
+
+namespace rocs {
+int lcb_validate_ext(const rocs_lcb_args* a, int64_t* C) { return lcb_validate(a, C); }
+int lcb_run_ext(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* body, cudaStream_t st, int* launches) {
+  return lcb_run(a, C, hdr, body, st, launches);
+}
+size_t lcb_body_bytes_ext(int64_t R, int64_t o_c, int64_t d) { return lcb_body(R, o_c, d).body; }
+int dca_validate_ext(const rocs_dca_args* a, int64_t* C, int64_t* T) { return dca_validate(a, C, T); }
+int dca_run_ext(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHeader* hdr, uint8_t* body,
+                cudaStream_t st, int* launches) {
+  return dca_run(a, C, T, n_units, hdr, body, st, launches);
+}
+size_t dca_body_bytes_ext(int64_t R, int64_t n_units) { return dca_body(R, n_units).body; }
+void set_last_launches(int n) { g_last_launches = n; }
+}  // namespace rocs
+
+extern "C" {
+
+size_t rocs_lcb_workspace_size(const rocs_lcb_args* a) {
+  int64_t C;
+  if (lcb_validate(a, &C) != ROCS_OK) return 0;
+  return lcb_bytes(a);
+}
+
+int rocs_lcb_forward(const rocs_lcb_args* a, rocs_stream_t stream) {
+  int64_t C = 0;
+  int rc = lcb_validate(a, &C);
+  if (rc) return rc;
+  if (!a->workspace || a->workspace_bytes < lcb_bytes(a) || (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ROCS_ERR_WORKSPACE;
+  int launches = 0;
+  WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
+  rc = lcb_run(a, C, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream), &launches);
+  if (rc == ROCS_OK) g_last_launches = launches;
+  return rc;
+}
+
+size_t rocs_dca_workspace_size(const rocs_dca_args* a) {
+  int64_t C, T;
+  if (dca_validate(a, &C, &T) != ROCS_OK) return 0;
+  return sizeof(WsHeader) + dca_body(a->R, dca_units(a)).body;
+}
+
+int rocs_dca_forward(const rocs_dca_args* a, rocs_stream_t stream) {
+  int64_t C = 0, T = 0;
+  int rc = dca_validate(a, &C, &T);
+  if (rc) return rc;
+  const int64_t n_units = dca_units(a);
+  if (!a->workspace || a->workspace_bytes < sizeof(WsHeader) + dca_body(a->R, n_units).body ||
+      (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ROCS_ERR_WORKSPACE;
+  int launches = 0;
+  WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
+  rc = dca_run(a, C, T, n_units, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream),
+               &launches);
+  if (rc == ROCS_OK) g_last_launches = launches;
+  return rc;
+}
+
+size_t rocs_proj_workspace_size(const rocs_proj_args* a) {
+  (void)a;
+  return sizeof(WsHeader);
+}
+
+int rocs_proj_forward(const rocs_proj_args* a, rocs_stream_t stream) {
+  if (!a || a->M < 0 || a->N <= 0 || a->K <= 0) return ROCS_ERR_INVALID_ARG;
+  if (a->N % 256 || a->K % 64) return ROCS_ERR_UNSUPPORTED;
+  if (a->M >= (int64_t(1) << 31) || a->N >= (int64_t(1) << 31) || a->K >= (int64_t(1) << 31))
+    return ROCS_ERR_UNSUPPORTED;
+  if (a->M > 0 && (!a->in || !a->w || !a->out || !al16(a->in) || !al16(a->w) || !al16(a->out)))
+    return ROCS_ERR_INVALID_ARG;
+  if (!a->workspace || a->workspace_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ROCS_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(a->workspace, 0, sizeof(WsHeader), st) != cudaSuccess) return ROCS_ERR_CUDA;
+  if (a->M == 0) {
+    g_last_launches = 0;
+    return ROCS_OK;
+  }
+  ProjParams p;
+  std::memset(&p, 0, sizeof(p));
+  bool ok = tmap_bf16(&p.tm_a, a->in, a->K, a->M, a->K * 2, 64, 128);
+  ok &= tmap_bf16(&p.tm_b, a->w, a->K, a->N, a->K * 2, 64, 256);
+  if (!ok) return ROCS_ERR_CUDA;
+  p.out = static_cast<__nv_bfloat16*>(a->out);
+  p.ws = static_cast<WsHeader*>(a->workspace);
+  p.M = (int)a->M;
+  p.N = (int)a->N;
+  p.K = (int)a->K;
+  const int64_t tiles = ((a->M + 127) / 128) * (a->N / 256);
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  if (launch_proj_sm100(p, grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  g_last_launches = 1;
+  return ROCS_OK;
+}
+
+int rocs_read_status(const void* workspace, rocs_stream_t stream, int32_t* device_code, int32_t* detail) {
+  if (!workspace || !device_code) return ROCS_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return ROCS_ERR_CUDA;
+  int32_t h[2] = {0, 0};
+  if (cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return ROCS_ERR_CUDA;
+  *device_code = h[0];
+  if (detail) *detail = h[1];
+  return ROCS_OK;
+}
+
+const char* rocs_status_string(int code) {
+  switch (code) {
+    case ROCS_OK: return "ROCS_OK";
+    case ROCS_ERR_INVALID_ARG: return "ROCS_ERR_INVALID_ARG";
+    case ROCS_ERR_BAD_OFFSETS: return "ROCS_ERR_BAD_OFFSETS";
+    case ROCS_ERR_UNSUPPORTED: return "ROCS_ERR_UNSUPPORTED";
+    case ROCS_ERR_CUDA: return "ROCS_ERR_CUDA";
+    case ROCS_ERR_TIMEOUT: return "ROCS_ERR_TIMEOUT";
+    case ROCS_ERR_WORKSPACE: return "ROCS_ERR_WORKSPACE";
+    case ROCS_ERR_DEVICE_INDEX: return "ROCS_ERR_DEVICE_INDEX";
+    default: return "unknown rocs_status";
+  }
+}
+
+int rocs_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

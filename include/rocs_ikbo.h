@@ -1,0 +1,209 @@
+/*
+ * rocs_ikbo.h -- C ABI of the B200 (sm_100a) In-Kernel Broadcast Optimization library.
+ *
+ * The operations are those of "ROCS: Request-Oriented Compute Sharing for
+ * Efficient Large-Scale Recommendation" (arXiv:2607.27744), as described in the
+ * paper-archivist reading notes of that paper:
+ *
+ *   IKBO-LCB  the two-group ROCSified linear compression block, section 3.1.2, Eq. (6)
+ *               Y^R   = W_RR . X^R
+ *               Y^C_i = W_CR . X^R_{m_i} + W_CC . X^C_i
+ *             executed as the section 4.1 decomposition, Eq. (14):
+ *               [Y^R ; Z] = [W_RR ; W_CR] . X^R        once per request (batch B_r)
+ *               Y^C_i     = Z_{m_i} + W_CC . X^C_i      per candidate, Z added in the
+ *                                                       GEMM epilogue (section 4.2.1)
+ *             with request and candidate tiles in one persistent kernel that waits on
+ *             per-request completion flags (section 4.2.3).
+ *   IKBO-DCA  candidate-group cross attention, section 3.2, Eq. (13):
+ *               A^C_i = softmax(scale . Q_i K_{m_i}^T) V_{m_i}     (non-causal)
+ *             with K/V stored once per request and m_i resolved inside the kernel
+ *             (section 4.3.1).
+ *   projection  the linear query generation of the chained block (section 3.2, Eq. (12),
+ *             read as a plain linear map): Q_i = W_q . vec(Y^C_i).
+ *
+ * Common conventions
+ *   - Every pointer named *_dev or any tensor pointer is a DEVICE pointer of the current
+ *     CUDA device; *_host pointers are host memory.  The caller owns every buffer; the
+ *     library never allocates, frees or synchronises inside a *_forward call, and all
+ *     device work is enqueued on `stream` (asynchronous w.r.t. the host).
+ *   - Tensors are dense row-major with the last axis contiguous.  bf16 tensors hold
+ *     IEEE bfloat16 bit patterns; accumulation is fp32; outputs are rounded once
+ *     (round-to-nearest-even) when stored.
+ *   - Candidate -> request association is a CSR offsets array cand_off[R+1]: request r
+ *     owns candidates cand_off[r] .. cand_off[r+1]-1 (candidates of a request are stored
+ *     contiguously, section 4.2.1).  m_i is derived from it.  Requests may own zero
+ *     candidates.  The host copy must equal the device copy.
+ *   - Host-side validation errors are returned synchronously and nothing is enqueued.
+ *     Device-side errors (a wait that exceeded its time limit, an index out of range)
+ *     are recorded in the workspace status word and reported by rocs_read_status().
+ *     No entry point calls exit/abort/__trap or lets a C++ exception cross the ABI.
+ *   - workspace: caller-allocated device memory of at least the *_workspace_size()
+ *     bytes, 256-byte aligned.  One workspace must not be used by two calls that can
+ *     run concurrently.  Each *_forward call resets the status word it uses.
+ */
+#ifndef ROCS_IKBO_H
+#define ROCS_IKBO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ROCS_API __attribute__((visibility("default")))
+#else
+#define ROCS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* rocs_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  ROCS_OK = 0,
+  ROCS_ERR_INVALID_ARG = 1, /* null pointer, negative size, misaligned pointer */
+  ROCS_ERR_BAD_OFFSETS = 2, /* CSR offsets not 0-based / not non-decreasing / wrong total */
+  ROCS_ERR_UNSUPPORTED = 3, /* shape outside the supported set (see each entry point) */
+  ROCS_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+  ROCS_ERR_TIMEOUT = 5,     /* device: a bounded wait expired (reported by rocs_read_status) */
+  ROCS_ERR_WORKSPACE = 6,   /* workspace missing or smaller than required */
+  ROCS_ERR_DEVICE_INDEX = 7 /* device: an index derived from device offsets fell out of range */
+} rocs_status;
+
+typedef enum { ROCS_F32 = 0, ROCS_BF16 = 1 } rocs_dtype;
+
+/* ------------------------------------------------------------------------------------
+ * IKBO-LCB  (section 3.1.2 Eq. (6); section 4.1 Eq. (14); sections 4.2.1-4.2.3)
+ *
+ *   x_req  [R, n_r, d]       request embeddings X^R (natural batch B_r = R)
+ *   x_cand [C, n_c, d]       candidate embeddings X^C (natural batch B_c = C)
+ *   w_rr   [o_r, n_r]        W_RR ;  w_cr [o_c, n_r] W_CR ;  w_cc [o_c, n_c] W_CC
+ *   y_req  [R, o_r, d]       out: Y^R (computed once per request)
+ *   y_cand [C, o_c, d]       out: Y^C
+ *   C = cand_off_host[R].
+ * dtype ROCS_BF16 (tcgen05 tensor-core path): n_r % 64 == 0, n_c in {64, 128},
+ *   d in {64, 128}, o_r % 128 == 0, o_c == 128; else ROCS_ERR_UNSUPPORTED.
+ * dtype ROCS_F32 (fp32 CUDA-core path, exact fp32 accumulation): any positive sizes
+ *   with n_r, n_c <= 1024 and d <= 1024.
+ * Row strides are d * sizeof(element) bytes; they must be multiples of 16 bytes
+ *   (the alignment contract of section 4.2.4; padding is the caller's), else
+ *   ROCS_ERR_UNSUPPORTED.  All tensor pointers must be 16-byte aligned.
+ * ---------------------------------------------------------------------------------- */
+typedef struct {
+  int64_t R;
+  int64_t n_r, n_c, d, o_r, o_c;
+  int32_t dtype; /* rocs_dtype, for all inputs and outputs */
+  const int32_t* cand_off_dev;  /* [R+1] */
+  const int32_t* cand_off_host; /* [R+1] */
+  const void* x_req;
+  const void* x_cand;
+  const void* w_rr;
+  const void* w_cr;
+  const void* w_cc;
+  void* y_req;
+  void* y_cand;
+  void* workspace; /* >= rocs_lcb_workspace_size(args) bytes: status, flags, tile counter, Z fp32 */
+  size_t workspace_bytes;
+} rocs_lcb_args;
+
+/* Bytes of workspace rocs_lcb_forward needs for these sizes (0 if the sizes are invalid). */
+ROCS_API size_t rocs_lcb_workspace_size(const rocs_lcb_args* args);
+
+/* IKBO-LCB forward.  One kernel launch (bf16) or two (fp32) plus one memset, on `stream`. */
+ROCS_API int rocs_lcb_forward(const rocs_lcb_args* args, rocs_stream_t stream);
+
+/* Explicit-expand baseline (ablation, not the method): materialises X^R per candidate
+ * into an expanded [C, n_r, d] tensor inside the workspace, then runs the same LCB
+ * kernels with the identity map (every candidate its own request), so Y^R and Z are
+ * recomputed per candidate.  y_req receives the request rows of the first candidate of
+ * each request; requests without candidates get W_RR . X^R computed on their own.
+ * Workspace: rocs_lcb_expand_workspace_size(). */
+ROCS_API size_t rocs_lcb_expand_workspace_size(const rocs_lcb_args* args);
+ROCS_API int rocs_lcb_forward_expand(const rocs_lcb_args* args, rocs_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * IKBO-DCA  (section 3.2 Eq. (13); section 4.3)
+ *
+ *   q_ptr  [C*q, H, dh] bf16   query tokens; candidate i owns rows i*q .. i*q+q-1
+ *   k_ptr  [T, H, dh]   bf16   request keys, T = seq_off_host[R]; request r owns rows
+ *   v_ptr  [T, H, dh]   bf16   seq_off[r] .. seq_off[r+1]-1 (stored once per request)
+ *   o_ptr  [C*q, H, dh] bf16   out: attention output
+ *   lse_ptr [C*q, H]    fp32   out (optional, may be NULL): natural-log sum-exp of the
+ *                              scaled scores; -inf where the request has no keys
+ *   scale                      softmax scale (1/sqrt(dh) in the usual setting)
+ * A request with keys but no candidates is legal (no work); a request with candidates
+ * but no keys gets O = 0 and LSE = -inf.  Every query token attends to all keys of its
+ * request (non-causal); query tokens of one candidate do not attend to each other.
+ * Supported: dh in {64, 128}, H >= 1, q >= 1, row strides multiples of 16 bytes.
+ * ---------------------------------------------------------------------------------- */
+typedef struct {
+  int64_t R, q, H, dh;
+  float scale;
+  const int32_t* cand_off_dev;  /* [R+1] */
+  const int32_t* cand_off_host; /* [R+1] */
+  const int32_t* seq_off_dev;   /* [R+1] */
+  const int32_t* seq_off_host;  /* [R+1] */
+  const void* q_ptr;
+  const void* k_ptr;
+  const void* v_ptr;
+  void* o_ptr;
+  float* lse_ptr;
+  void* workspace; /* >= rocs_dca_workspace_size(args): status, work-unit table, counter */
+  size_t workspace_bytes;
+} rocs_dca_args;
+
+ROCS_API size_t rocs_dca_workspace_size(const rocs_dca_args* args);
+
+/* IKBO-DCA forward: a scheduling kernel (work-unit table, longest request first) and the
+ * persistent attention kernel, both on `stream`. */
+ROCS_API int rocs_dca_forward(const rocs_dca_args* args, rocs_stream_t stream);
+
+/* Explicit-expand baseline (ablation): copies each candidate's request K/V into a
+ * per-candidate buffer (the materialised broadcast of section 4.3), `chunk` candidates
+ * at a time, and runs the same attention kernel with the identity map on each chunk.
+ * Workspace: rocs_dca_expand_workspace_size(args, chunk). */
+ROCS_API size_t rocs_dca_expand_workspace_size(const rocs_dca_args* args, int64_t chunk);
+ROCS_API int rocs_dca_forward_expand(const rocs_dca_args* args, int64_t chunk, rocs_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Linear query projection of the chained block (section 3.2, Eq. (12), plain linear
+ * map, no bias, no activation):  out[i, :] = W . in[i, :]
+ *   in  [M, K] bf16 (for the chained block: Y^C viewed as [C, o_c*d])
+ *   w   [N, K] bf16
+ *   out [M, N] bf16
+ * Supported: K % 64 == 0, N % 256 == 0, M >= 0.
+ * ---------------------------------------------------------------------------------- */
+typedef struct {
+  int64_t M, N, K;
+  const void* in;
+  const void* w;
+  void* out;
+  void* workspace; /* >= rocs_proj_workspace_size(args) */
+  size_t workspace_bytes;
+} rocs_proj_args;
+
+ROCS_API size_t rocs_proj_workspace_size(const rocs_proj_args* args);
+ROCS_API int rocs_proj_forward(const rocs_proj_args* args, rocs_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * Status and introspection
+ * ---------------------------------------------------------------------------------- */
+
+/* Synchronises `stream`, then reads the device status word of `workspace` (the workspace
+ * of the last *_forward call that used it) into *device_code (a rocs_status) and, if
+ * `detail` is non-NULL, a code naming where the error was raised.  Returns ROCS_OK or
+ * ROCS_ERR_CUDA / ROCS_ERR_INVALID_ARG for the read itself. */
+ROCS_API int rocs_read_status(const void* workspace, rocs_stream_t stream, int32_t* device_code, int32_t* detail);
+
+/* Human-readable name of a rocs_status value (static string). */
+ROCS_API const char* rocs_status_string(int code);
+
+/* Number of kernel launches the last successful *_forward call on this host thread
+ * enqueued (memsets not counted). */
+ROCS_API int rocs_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROCS_IKBO_H */

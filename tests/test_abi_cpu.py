@@ -1,0 +1,110 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the header declares,
+and rejects malformed arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from attention_ikbo_b200.build import build
+
+    build()
+    import attention_ikbo_b200 as m
+
+    return m.load_library()
+
+
+def declared_symbols():
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        names.update(re.findall(r"ROCS_API\s+[\w\s\*]+?\b(rocs_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    lib.rocs_status_string.restype = ctypes.c_char_p
+    assert lib.rocs_status_string(0) == b"ROCS_OK"
+    assert lib.rocs_status_string(5) == b"ROCS_ERR_TIMEOUT"
+
+
+def _lcb_args(m, off, n_c=64, dtype=1, d=128, ws_bytes=0):
+    off = np.asarray(off, np.int32)
+    fake = 0x10000  # aligned non-null placeholders: validation fails before any dereference
+    a = m._binding.LcbArgs(R=len(off) - 1, n_r=256, n_c=n_c, d=d, o_r=128, o_c=128, dtype=dtype,
+                           cand_off_dev=fake, cand_off_host=off.ctypes.data, x_req=fake, x_cand=fake, w_rr=fake,
+                           w_cr=fake, w_cc=fake, y_req=fake, y_cand=fake, workspace=fake if ws_bytes else None,
+                           workspace_bytes=ws_bytes)
+    return a, off
+
+
+def test_lcb_host_validation(lib):
+    import attention_ikbo_b200 as m
+
+    a, keep = _lcb_args(m, [0, 3, 2, 6])
+    assert lib.rocs_lcb_workspace_size(ctypes.byref(a)) == 0
+    assert lib.rocs_lcb_forward(ctypes.byref(a), None) == 2  # ROCS_ERR_BAD_OFFSETS
+    a, keep = _lcb_args(m, [1, 3])
+    assert lib.rocs_lcb_forward(ctypes.byref(a), None) == 2
+    a, keep = _lcb_args(m, [0, 3, 6], n_c=48)
+    assert lib.rocs_lcb_forward(ctypes.byref(a), None) == 3  # ROCS_ERR_UNSUPPORTED (n_c)
+    a, keep = _lcb_args(m, [0, 3, 6], d=100)
+    assert lib.rocs_lcb_forward(ctypes.byref(a), None) == 3  # 200-byte rows break the 16-byte contract
+    a, keep = _lcb_args(m, [0, 3, 6])
+    need = lib.rocs_lcb_workspace_size(ctypes.byref(a))
+    # header 256 + flags (2 ints, padded to 256) + Z 2 x 128 x 128 fp32
+    assert need == 256 + 256 + 2 * 128 * 128 * 4
+    a, keep = _lcb_args(m, [0, 3, 6], ws_bytes=need - 1)
+    assert lib.rocs_lcb_forward(ctypes.byref(a), None) == 6  # ROCS_ERR_WORKSPACE
+    a.x_req = 0x10008  # misaligned
+    assert lib.rocs_lcb_forward(ctypes.byref(a), None) == 1
+
+
+def test_dca_host_validation(lib):
+    import attention_ikbo_b200 as m
+
+    co = np.array([0, 2, 5], np.int32)
+    so = np.array([0, 7, 6], np.int32)
+    fake = 0x20000
+    a = m._binding.DcaArgs(R=2, q=1, H=2, dh=128, scale=0.1, cand_off_dev=fake, cand_off_host=co.ctypes.data,
+                           seq_off_dev=fake, seq_off_host=so.ctypes.data, q_ptr=fake, k_ptr=fake, v_ptr=fake,
+                           o_ptr=fake, lse_ptr=None, workspace=None, workspace_bytes=0)
+    assert lib.rocs_dca_forward(ctypes.byref(a), None) == 2
+    so[2] = 9
+    assert lib.rocs_dca_forward(ctypes.byref(a), None) == 6  # valid, but no workspace
+    # 2 requests x 2 heads x ceil(rows/256) units = 4 units of 16 B after 256 + pad(3R+1 ints)
+    assert lib.rocs_dca_workspace_size(ctypes.byref(a)) == 256 + 256 + 4 * 16
+    a.dh = 96
+    assert lib.rocs_dca_forward(ctypes.byref(a), None) == 3
+
+
+def test_proj_host_validation(lib):
+    import attention_ikbo_b200 as m
+
+    a = m._binding.ProjArgs(M=10, N=200, K=64, in_=0x1000, w=0x1000, out=0x1000, workspace=None, workspace_bytes=0)
+    assert lib.rocs_proj_forward(ctypes.byref(a), None) == 3
+    a.N = 256
+    assert lib.rocs_proj_forward(ctypes.byref(a), None) == 6
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import attention_ikbo_b200._binding as b
+
+    monkeypatch.setattr(b, "_lib", None)
+    monkeypatch.setattr(b, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        b.load_library()

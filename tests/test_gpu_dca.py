@@ -1,0 +1,117 @@
+"""IKBO-DCA on the GPU (through the C ABI) against the fp64 oracle.
+
+Operation: ROCS (arXiv:2607.27744), section 3.2 Eq. (13), candidate cross attention
+over K/V stored once per request, m_i resolved in the kernel (section 4.3.1).
+"""
+import numpy as np
+import pytest
+import torch
+
+import rocs_inputs as ri
+from _helpers import assert_close, dev, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ikbo():
+    import attention_ikbo_b200 as m
+
+    m.load_library()
+    return m
+
+
+def run_dca(ikbo, x, expand_chunk=None):
+    o, lse = ikbo.rocs_dca_forward(dev(x.q_t), dev(x.k_t), dev(x.v_t), x.cand_off, x.seq_off, x.q, x.scale,
+                                   expand_chunk=expand_chunk)
+    code, detail = ikbo.rocs_read_status(ikbo.rocs_dca_forward.last_workspace)
+    assert code == 0, f"device status {ikbo.STATUS_NAMES.get(code)} at {detail}"
+    return o, lse
+
+
+def check(oracle_mod, x, o, lse, sel=None):
+    sel = np.arange(x.C) if sel is None else np.asarray(sel)
+    oo, ll = oracle_mod.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, x.v_t, x.q, x.scale, sel_cand=sel)
+    rows = (sel[:, None] * x.q + np.arange(x.q)[None, :]).ravel()
+    ridx = torch.as_tensor(rows, device=o.device)
+    got_o = host_f64(o[ridx]).reshape(oo.shape)
+    assert_close(got_o, oo, "bf16", "O")
+    got_l = host_f64(lse[ridx]).reshape(ll.shape)
+    fin = np.isfinite(ll)
+    assert np.array_equal(np.isfinite(got_l), fin)
+    assert np.all(got_l[~fin] == -np.inf)
+    if fin.any():
+        assert_close(got_l[fin], ll[fin], "bf16", "LSE")
+
+
+CASES = [  # (counts, lengths, q, H, dh)
+    ([2, 5, 0], [5, 300, 17], 2, 2, 128),
+    ([200, 1, 0, 513], [1, 129, 700, 128], 1, 3, 64),
+    ([64, 70], [1000, 257], 4, 1, 128),
+    ([3, 300], [128, 2049], 1, 4, 64),
+]
+
+
+@pytest.mark.parametrize("counts,lengths,q,H,dh", CASES)
+def test_dca_small(ikbo, oracle_mod, counts, lengths, q, H, dh):
+    x = ri.make_dca("t", counts, lengths, q, H, dh, 17 + q + H + dh)
+    o, lse = run_dca(ikbo, x)
+    check(oracle_mod, x, o, lse)
+
+
+def test_dca_empty_keys(ikbo, oracle_mod):
+    x = ri.make_dca("t", [3, 4, 2], [0, 50, 0], 2, 2, 64, 5)
+    o, lse = run_dca(ikbo, x)
+    check(oracle_mod, x, o, lse)
+
+
+def test_dca_index_probe(ikbo):
+    """V of request r is constant r  ->  every output of candidate i rounds to m_i."""
+    counts, lengths = [3, 0, 260, 1, 7], [40, 9, 300, 1, 129]
+    x = ri.make_dca("t", counts, lengths, 2, 2, 128, 8)
+    v = np.zeros(x.v_t.shape, np.float32)
+    for r in range(x.R):
+        v[x.seq_off[r]: x.seq_off[r + 1]] = r
+    x.v_t = (v.view(np.uint32) >> 16).astype(np.uint16)
+    o, _ = run_dca(ikbo, x)
+    m = np.repeat(np.arange(x.R), counts)
+    got = np.rint(host_f64(o)).reshape(x.C, -1)
+    assert np.array_equal(got, np.broadcast_to(m[:, None].astype(np.float64), got.shape))
+
+
+def test_dca_permutation_within_request(ikbo, oracle_mod):
+    x = ri.make_dca("t", [100, 40], [300, 77], 1, 2, 128, 12)
+    o0, _ = run_dca(ikbo, x)
+    perm = np.concatenate([np.random.RandomState(3).permutation(100), 100 + np.random.RandomState(4).permutation(40)])
+    x.q_t = np.ascontiguousarray(x.q_t.reshape(x.C, x.q, x.H, x.dh)[perm].reshape(x.q_t.shape))
+    o1, _ = run_dca(ikbo, x)
+    assert_close(host_f64(o1), host_f64(o0)[perm], "bf16", "permuted O")
+
+
+def test_dca_expand_baseline_matches(ikbo, oracle_mod):
+    x = ri.make_dca("t", [5, 0, 9, 2], [130, 4, 64, 0], 2, 2, 128, 19)
+    o, lse = run_dca(ikbo, x, expand_chunk=4)
+    check(oracle_mod, x, o, lse)
+
+
+def _sample(x, n, seed):
+    rs = np.random.RandomState(seed)
+    sel = set(rs.choice(x.C, size=min(n, x.C), replace=False).tolist())
+    for r in range(x.R):
+        if x.cand_off[r + 1] > x.cand_off[r]:
+            sel.update([int(x.cand_off[r]), int(x.cand_off[r + 1]) - 1])
+    return np.array(sorted(sel), dtype=np.int64)
+
+
+def test_dca_bf16_full_size_sampled(ikbo, oracle_mod):
+    """R=32, L=2048, H=8, dh=128, 512 candidates per request, q=1."""
+    x = ri.dca_bf16()
+    o, lse = run_dca(ikbo, x)
+    check(oracle_mod, x, o, lse, sel=_sample(x, 64, 2))
+
+
+def test_dca_long_full_size_sampled(ikbo, oracle_mod):
+    """R=8, L_r~U{4096..8192}, H=4, dh=128, 2048 candidates per request, q=4."""
+    x = ri.dca_long()
+    o, lse = run_dca(ikbo, x)
+    check(oracle_mod, x, o, lse, sel=_sample(x, 24, 3))
