@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     last_launch_count,
     lib_path,
     load_library,
+    offsets,
     rocs_dca_forward,
     rocs_dca_forward_expand,
     rocs_lcb_forward,

@@ -89,8 +89,18 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def offsets(off, device="cuda"):
+    """CSR offsets as the pair the C ABI needs: (device int32 tensor, host int32 numpy array).
+
+    Pass the returned pair back into the forward functions to avoid a host<->device copy per call.
+    """
+    return _offsets(off, torch.device(device))
+
+
 def _offsets(off, device):
-    """(device int32 tensor, host int32 numpy array) from a tensor / array / list."""
+    """(device int32 tensor, host int32 numpy array) from a pair, a tensor, an array or a list."""
+    if isinstance(off, tuple) and len(off) == 2:
+        return off
     if isinstance(off, torch.Tensor):
         host = off.detach().to("cpu", torch.int32).contiguous().numpy()
         dev = off if (off.is_cuda and off.dtype == torch.int32 and off.is_contiguous()) else \

@@ -1,0 +1,615 @@
+#!/usr/bin/env python
+"""Benchmark of the IKBO hot path on B200 (one JSON line on rank 0).
+
+A step is one pass of the hot path over one batch of synthetic inputs.  Default workload
+("ikbo_step"): IKBO-LCB on the bf16 LCB workload (R=64 requests, N_r ~ U{256..1024},
+n_r=256, n_c=64, d=128, o_r=o_c=128) followed by IKBO-DCA on the long-history workload
+(R=8, L_r ~ U{4096..8192}, H=4, dh=128, 2048 candidates x q=4 per request).  Other
+workloads: "lcb", "dca", "dca_short" (R=32, L=2048, H=8, 512 candidates, q=1) and "chain"
+(LCB -> query projection -> DCA, lognormal candidates per request).
+
+Reported: TFLOP/s on the non-materialised IKBO formulation (value), per-kernel rooflines
+against MEASURED_PEAKS.json, an end-to-end figure with host<->device copies, the fp64 CPU
+oracle as the CPU baseline, launches and SM clocks sampled during the timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload W] [--impl ikbo|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import rocs_inputs as ri  # noqa: E402
+from attention_ikbo_b200 import accounting as acc  # noqa: E402
+
+METRIC = "IKBO LCB/DCA TFLOP/s & candidates/s at 1 B200; % of bf16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SRC = {"lcb": "attention_ikbo_b200/csrc/lcb_sm100.cu", "dca": "attention_ikbo_b200/csrc/dca_sm100.cu",
+              "proj": "attention_ikbo_b200/csrc/proj_sm100.cu"}
+
+
+# ----------------------------------------------------------------------------------- parts
+class Part:
+    name = ""
+    bound = "hbm"
+    kernel = ""
+
+    def flops(self):
+        raise NotImplementedError
+
+    def bytes(self):
+        raise NotImplementedError
+
+
+class LcbPart(Part):
+    bound, kernel = "hbm", "lcb"
+
+    def __init__(self, x: ri.LcbInputs, name="lcb"):
+        self.x, self.name = x, name
+        self.units = x.C
+
+    def dims(self):
+        x = self.x
+        return x.R, x.C, x.n_r, x.n_c, x.d, x.o_r, x.o_c
+
+    def flops(self):
+        return acc.lcb_flops(*self.dims())
+
+    def bytes(self):
+        return acc.lcb_bytes(*self.dims())
+
+    # -- GPU
+    def to_device(self, ikbo, torch, dev):
+        x = self.x
+        self.h_in = [_pin(torch, a) for a in (x.x_req, x.x_cand)]
+        self.d_in = [h.to(dev) for h in self.h_in]
+        self.d_w = [_to_dev(torch, a, dev) for a in (x.w_rr, x.w_cr, x.w_cc)]
+        self.off = ikbo.offsets(x.cand_off, dev)
+        self.h_off = _pin(torch, x.cand_off)
+        self.y_req = torch.empty((x.R, x.o_r, x.d), dtype=torch.bfloat16, device=dev)
+        self.y_cand = torch.empty((x.C, x.o_c, x.d), dtype=torch.bfloat16, device=dev)
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (self.y_req, self.y_cand)]
+        ikbo.rocs_lcb_forward(*self.d_in, *self.d_w, self.off, self.y_req, self.y_cand)
+        self.ws = ikbo.rocs_lcb_forward.last_workspace
+
+    def run(self, ikbo):
+        ikbo.rocs_lcb_forward(*self.d_in, *self.d_w, self.off, self.y_req, self.y_cand, workspace=self.ws)
+        return ikbo.last_launch_count()
+
+    def h2d(self):
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+        self.off[0].copy_(self.h_off, non_blocking=True)
+        return sum(h.numel() * h.element_size() for h in self.h_in) + self.h_off.numel() * 4
+
+    def d2h(self):
+        for h, d in zip(self.h_out, (self.y_req, self.y_cand)):
+            h.copy_(d, non_blocking=True)
+        return sum(h.numel() * h.element_size() for h in self.h_out)
+
+    def status(self, ikbo):
+        return ikbo.rocs_read_status(self.ws)
+
+    # -- CPU oracle on a sample of candidates; returns seconds for the sample and the fraction it covers
+    def oracle_sample(self, oracle, n, seed):
+        x = self.x
+        rs = np.random.RandomState(seed)
+        sel = rs.choice(x.C, size=min(n, x.C), replace=False)
+        t0 = time.perf_counter()
+        oracle.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, sel_req=[], sel_cand=sel)
+        return time.perf_counter() - t0, len(sel) / x.C
+
+
+class DcaPart(Part):
+    bound, kernel = "tensor", "dca"
+
+    def __init__(self, x: ri.DcaInputs, name="dca"):
+        self.x, self.name = x, name
+        self.units = x.C
+
+    def flops(self):
+        x = self.x
+        return acc.dca_flops(x.cand_off, x.seq_off, x.q, x.H, x.dh)
+
+    def bytes(self):
+        x = self.x
+        return acc.dca_bytes(x.C, x.total_L, x.q, x.H, x.dh)
+
+    def to_device(self, ikbo, torch, dev, q_dev=None):
+        x = self.x
+        self.h_in = [_pin(torch, a) for a in ((x.q_t,) if q_dev is None else ()) + (x.k_t, x.v_t)]
+        d_in = [h.to(dev) for h in self.h_in]
+        if q_dev is None:
+            self.q_dev, self.k_dev, self.v_dev = d_in
+        else:
+            self.q_dev = q_dev
+            self.k_dev, self.v_dev = d_in
+        self.d_in = d_in
+        self.coff = ikbo.offsets(x.cand_off, dev)
+        self.soff = ikbo.offsets(x.seq_off, dev)
+        self.h_offs = [_pin(torch, x.cand_off), _pin(torch, x.seq_off)]
+        self.o = torch.empty((x.C * x.q, x.H, x.dh), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((x.C * x.q, x.H), dtype=torch.float32, device=dev)
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (self.o, self.lse)]
+        ikbo.rocs_dca_forward(self.q_view(), self.k_dev, self.v_dev, self.coff, self.soff, x.q, x.scale, self.o,
+                              self.lse)
+        self.ws = ikbo.rocs_dca_forward.last_workspace
+
+    def q_view(self):
+        x = self.x
+        return self.q_dev.view(x.C * x.q, x.H, x.dh)
+
+    def run(self, ikbo):
+        x = self.x
+        ikbo.rocs_dca_forward(self.q_view(), self.k_dev, self.v_dev, self.coff, self.soff, x.q, x.scale, self.o,
+                              self.lse, workspace=self.ws)
+        return ikbo.last_launch_count()
+
+    def h2d(self):
+        n = 0
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+            n += h.numel() * h.element_size()
+        for h, d in zip(self.h_offs, (self.coff[0], self.soff[0])):
+            d.copy_(h, non_blocking=True)
+            n += h.numel() * 4
+        return n
+
+    def d2h(self):
+        for h, d in zip(self.h_out, (self.o, self.lse)):
+            h.copy_(d, non_blocking=True)
+        return sum(h.numel() * h.element_size() for h in self.h_out)
+
+    def status(self, ikbo):
+        return ikbo.rocs_read_status(self.ws)
+
+    def oracle_sample(self, oracle, n, seed):
+        x = self.x
+        rs = np.random.RandomState(seed)
+        sel = rs.choice(x.C, size=min(n, x.C), replace=False)
+        # fraction of the algorithmic work the sample covers (candidates differ by their request's L_r)
+        L = np.diff(x.seq_off.astype(np.int64))
+        m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+        frac = float(L[m[sel]].sum()) / float(L[m].sum())
+        t0 = time.perf_counter()
+        oracle.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, x.v_t, x.q, x.scale, sel_cand=sel)
+        return time.perf_counter() - t0, frac
+
+
+class ProjPart(Part):
+    bound, kernel = "tensor", "proj"
+
+    def __init__(self, ci: ri.ChainInputs, lcb_part: LcbPart):
+        self.ci, self.lcb, self.name = ci, lcb_part, "proj"
+        self.M, self.K = ci.lcb.C, ci.lcb.o_c * ci.lcb.d
+        self.N = ci.H * ci.dh
+        self.units = self.M
+
+    def flops(self):
+        return acc.proj_flops(self.M, self.N, self.K)
+
+    def bytes(self):
+        return acc.proj_bytes(self.M, self.N, self.K)
+
+    def to_device(self, ikbo, torch, dev):
+        self.w = _to_dev(torch, self.ci.w_q, dev)
+        self.out = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
+        ikbo.rocs_proj_forward(self.lcb.y_cand.view(self.M, -1), self.w, self.out)
+        self.ws = ikbo.rocs_proj_forward.last_workspace
+        self.h_out = []
+
+    def run(self, ikbo):
+        ikbo.rocs_proj_forward(self.lcb.y_cand.view(self.M, -1), self.w, self.out, workspace=self.ws)
+        return ikbo.last_launch_count()
+
+    def h2d(self):
+        return 0
+
+    def d2h(self):
+        return 0
+
+    def status(self, ikbo):
+        return ikbo.rocs_read_status(self.ws)
+
+    def oracle_sample(self, oracle, n, seed):
+        ci = self.ci
+        rs = np.random.RandomState(seed)
+        sel = rs.choice(self.M, size=min(n, self.M), replace=False)
+        y = ri.normal(seed, 99, (len(sel), self.K))  # the projection's cost does not depend on the values
+        t0 = time.perf_counter()
+        oracle.proj(y, ci.w_q)
+        return time.perf_counter() - t0, len(sel) / self.M
+
+
+def _pin(torch, a):
+    t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16 else np.ascontiguousarray(a))
+    if a.dtype == np.uint16:
+        t = t.view(torch.bfloat16)
+    return t.pin_memory()
+
+
+def _to_dev(torch, a, dev):
+    return _pin(torch, a).to(dev)
+
+
+class ChainOracle:
+    """CPU oracle of the chained block on sampled candidates (all three stages per candidate)."""
+
+    name = "chain"
+
+    def __init__(self, ci):
+        self.ci = ci
+
+    def oracle_sample(self, oracle, n, seed):
+        ci = self.ci
+        C = ci.lcb.C
+        sel = np.random.RandomState(seed).choice(C, size=min(n, C), replace=False)
+        L = np.diff(ci.seq_off.astype(np.int64))
+        m = np.repeat(np.arange(ci.lcb.R), np.diff(ci.lcb.cand_off))
+        # LCB + projection cost is the same per candidate, DCA cost scales with L_{m_i}
+        x = ci.lcb
+        w_fixed = acc.lcb_candidate_flops(x.n_c, x.d, x.o_c) + acc.proj_flops(1, ci.H * ci.dh, x.o_c * x.d)
+        w_dca = 4 * ci.H * ci.dh * L[m]
+        frac = float((w_fixed + w_dca[sel]).sum()) / float((w_fixed + w_dca).sum())
+        t0 = time.perf_counter()
+        oracle.chain(ci, sel)
+        return time.perf_counter() - t0, frac
+
+
+_CHAIN = {}
+
+
+def oracle_parts(workload, parts):
+    return [ChainOracle(_CHAIN["ci"])] if workload == "chain" else parts
+
+
+def make_parts(workload):
+    if workload == "ikbo_step":
+        return [LcbPart(ri.lcb_bf16()), DcaPart(ri.dca_long())]
+    if workload == "lcb":
+        return [LcbPart(ri.lcb_bf16())]
+    if workload == "dca":
+        return [DcaPart(ri.dca_long())]
+    if workload == "dca_short":
+        return [DcaPart(ri.dca_bf16())]
+    if workload == "chain":
+        ci = ri.chain()
+        lcb = LcbPart(ci.lcb, "chain_lcb")
+        x = ci.lcb
+        qdummy = np.zeros((0,), np.uint16)
+        dca_in = ri.DcaInputs("chain_dca", x.cand_off, ci.seq_off, 1, ci.H, ci.dh, ci.scale, qdummy, ci.k_t, ci.v_t)
+        _CHAIN["ci"] = ci
+        return [lcb, ProjPart(ci, lcb), DcaPart(dca_in, "chain_dca")]
+    raise ValueError(workload)
+
+
+def workload_config(workload, parts):
+    if workload == "chain":
+        ci = _CHAIN["ci"]
+        return {"workload": "chain", "recipe": ci.recipe, "R": ci.lcb.R, "C": ci.lcb.C, "sum_L": int(ci.seq_off[-1])}
+    cfg = {"workload": workload, "parts": {}}
+    for p in parts:
+        x = p.x
+        if isinstance(p, LcbPart):
+            cfg["parts"][p.name] = {"R": x.R, "C": x.C, "n_r": x.n_r, "n_c": x.n_c, "d": x.d, "o_r": x.o_r,
+                                    "o_c": x.o_c, "recipe": x.recipe}
+        else:
+            cfg["parts"][p.name] = {"R": x.R, "C": x.C, "q": x.q, "H": x.H, "dh": x.dh, "sum_L": x.total_L,
+                                    "recipe": x.recipe}
+    return cfg
+
+
+# ----------------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sha(kernel):
+    h = hashlib.sha256()
+    for rel in (KERNEL_SRC[kernel], "attention_ikbo_b200/csrc/sm100.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, units):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f).get(kernel)
+    if not d or d.get("src_sha") != kernel_sha(kernel):
+        return None
+    return d["dram_bytes_per_unit"] * units
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", gpu_id], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+def reduce_max(x: float, dist, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------------- arms
+def cpu_baseline(parts, oracle, budget_s=12.0):
+    """fp64 oracle on a bounded random sample of each part, scaled to the full step."""
+    est = 0.0
+    desc = []
+    for i, p in enumerate(parts):
+        t1, f1 = p.oracle_sample(oracle, 2, 100 + i)  # calibration
+        per = max(t1 / max(f1, 1e-12), 1e-9)  # seconds for the whole part
+        unit_time = t1 / 2
+        n = int(max(2, min(4096, (budget_s / len(parts)) / max(unit_time, 1e-6))))
+        t, f = p.oracle_sample(oracle, n, 200 + i)
+        est += t / f
+        desc.append(f"{p.name}: {n} random candidates ({100 * f:.3f}% of the part) in {t:.1f} s")
+        del per
+    return est, "; ".join(desc)
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, each step a bounded sample of the workload."""
+    import oracle
+
+    oracle.build_lib()
+    parts = make_parts(args.workload)
+    step_flops = sum(p.flops() for p in parts)
+    oparts = oracle_parts(args.workload, parts)
+    per_step_budget = max(0.05, 150.0 / max(1, args.steps + args.warmup))
+    unit_t = []
+    for i, p in enumerate(oparts):
+        t, f = p.oracle_sample(oracle, 1, 7 + i)
+        unit_t.append(t)
+    ns = [int(max(1, min(4096, per_step_budget / len(oparts) / max(t, 1e-6)))) for t in unit_t]
+    vals, times = [], []
+    for k in range(args.warmup + args.steps):
+        est = 0.0
+        for i, p in enumerate(oparts):
+            t, f = p.oracle_sample(oracle, ns[i], 1000 * k + i)
+            est += t / f
+        if k >= args.warmup:
+            times.append(est)
+            vals.append(step_flops / est / 1e12)
+    value = float(statistics.mean(vals))
+    sample = "; ".join(f"{p.name}: {n} random candidates per step, scaled by the work they cover"
+                       for p, n in zip(oparts, ns))
+    cores = oracle.max_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(statistics.mean(times)),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(args.workload, parts),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def run_ikbo(args):
+    import torch
+
+    import attention_ikbo_b200 as ikbo
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    ikbo.load_library()
+
+    parts = make_parts(args.workload)
+    for p in parts:
+        if isinstance(p, DcaPart) and args.workload == "chain":
+            p.to_device(ikbo, torch, dev, q_dev=parts[1].out)
+        else:
+            p.to_device(ikbo, torch, dev)
+    torch.cuda.synchronize()
+    for p in parts:
+        code, detail = p.status(ikbo)
+        if code != 0:
+            raise SystemExit(f"{p.name}: device status {ikbo.STATUS_NAMES.get(code)} at {detail}")
+
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # 256 MiB > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def step():
+        n = 0
+        for p in parts:
+            n += p.run(ikbo)
+        return n
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = None if args.no_clocks else ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    if sampler is not None:
+        time.sleep(0.3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(args.steps)]
+    launches = 0
+    for k in range(args.steps):
+        flush.zero_()  # L2 flush between steps, outside the per-step events
+        ev[k][0].record(stream)
+        for j, p in enumerate(parts):
+            launches += p.run(ikbo)
+            ev[k][j + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler is not None else None
+
+    part_ms = [statistics.mean(ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(args.steps))
+               for j in range(len(parts))]
+    step_ms = sum(part_ms)
+    for p in parts:
+        code, detail = p.status(ikbo)
+        if code != 0:
+            raise SystemExit(f"{p.name}: device status {ikbo.STATUS_NAMES.get(code)} at {detail}")
+    step_ms = reduce_max(step_ms, dist, dev)
+
+    # ---- end to end through the public API: pinned host inputs -> device -> kernels -> host outputs
+    e2e = None
+    if not args.no_e2e:
+        h2d = d2h = 0
+        for _ in range(2):
+            for p in parts:
+                p.h2d()
+            step()
+            for p in parts:
+                p.d2h()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            h2d = sum(p.h2d() for p in parts)
+            step()
+            d2h = sum(p.d2h() for p in parts)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        e2e_ms = reduce_max(e2e_ms, dist, dev)
+        step_flops_ = sum(p.flops() for p in parts)
+        e2e = {"value": world * step_flops_ / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    step_flops = sum(p.flops() for p in parts)
+    value = world * step_flops / (step_ms * 1e-3) / 1e12
+    rooflines, part_rows = [], []
+    for p, ms in zip(parts, part_ms):
+        sec = ms * 1e-3
+        if p.bound == "hbm":
+            ach, peak, unit = p.bytes() / sec / 1e9, peaks["hbm_gbs"], "GB/s"
+        else:
+            ach, peak, unit = p.flops() / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        rf = {"kernel": p.name, "bound": p.bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+              "traffic": ncu_traffic(p.kernel, p.units), "peak_source": f"{peak_src} (burst)"}
+        rooflines.append(rf)
+        part_rows.append({"name": p.name, "ms": ms, "tflops": p.flops() / sec / 1e12, "gbs": p.bytes() / sec / 1e9,
+                          "candidates_per_s": p.units / sec, "algorithmic_flops": p.flops(),
+                          "algorithmic_bytes": p.bytes()})
+    dom = max(range(len(parts)), key=lambda j: part_ms[j])
+
+    cpu = None
+    if not args.no_cpu:
+        import oracle
+
+        oracle.build_lib()
+        est_s, sample = cpu_baseline(oracle_parts(args.workload, parts), oracle, args.cpu_budget)
+        cpu = {"value": step_flops / est_s / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+               "sample": sample, "est_seconds_per_step": est_s}
+
+    cfg = workload_config(args.workload, parts)
+    cfg.update({"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "l2": "flushed between timed steps (256 MiB write outside the per-step CUDA events)"})
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "roofline": {k: v for k, v in rooflines[dom].items()}, "rooflines": rooflines, "parts": part_rows,
+            "candidates_per_s": {r["name"]: r["candidates_per_s"] for r in part_rows},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ikbo", choices=["ikbo", "reference"])
+    ap.add_argument("--workload", default="ikbo_step", choices=["ikbo_step", "lcb", "dca", "dca_short", "chain"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for the CPU baseline")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        run_reference(args)
+    else:
+        run_ikbo(args)
+
+
+if __name__ == "__main__":
+    main()
