@@ -63,6 +63,7 @@ def load_library():
             getattr(lib, name).restype = _sz
             getattr(lib, name).argtypes = argt
         for name, argt in [("rocs_lcb_forward", [P(LcbArgs), _vp]), ("rocs_lcb_forward_expand", [P(LcbArgs), _vp]),
+                           ("rocs_lcb_forward_noalloc", [P(LcbArgs), _vp]),
                            ("rocs_dca_forward", [P(DcaArgs), _vp]), ("rocs_proj_forward", [P(ProjArgs), _vp]),
                            ("rocs_dca_forward_expand", [P(DcaArgs), _i64, _vp]),
                            ("rocs_read_status", [_vp, _vp, P(_i32), P(_i32)])]:
@@ -163,6 +164,19 @@ def rocs_lcb_forward(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req=None, y_ca
     fn = lib.rocs_lcb_forward_expand if expand else lib.rocs_lcb_forward
     _check(fn(ctypes.byref(a), _stream(stream)), fn.__name__)
     rocs_lcb_forward.last_workspace = ws
+    return y_req, y_cand
+
+
+def rocs_lcb_forward_noalloc(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y_cand, stream=None):
+    """IKBO-LCB without a workspace, for callers that cannot allocate device memory.
+
+    Uses the library's fixed device scratch array instead of a workspace (see the header for its
+    size limit and for why concurrent calls on one device must be serialised).  ``y_req`` and
+    ``y_cand`` must be given: this call allocates nothing.
+    """
+    lib = load_library()
+    a, keep, y_req, y_cand = _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y_cand)
+    _check(lib.rocs_lcb_forward_noalloc(ctypes.byref(a), _stream(stream)), "rocs_lcb_forward_noalloc")
     return y_req, y_cand
 
 

@@ -121,6 +121,27 @@ ROCS_API int rocs_lcb_forward(const rocs_lcb_args* args, rocs_stream_t stream);
 ROCS_API size_t rocs_lcb_expand_workspace_size(const rocs_lcb_args* args);
 ROCS_API int rocs_lcb_forward_expand(const rocs_lcb_args* args, rocs_stream_t stream);
 
+/* IKBO-LCB without a caller workspace.  The paper has no counterpart: this entry point
+ * exists for callers that cannot hand the library device memory -- e.g. a plugin inside a
+ * serving process whose device memory is fully reserved by the host framework's own pool
+ * with no allocator exposed, or a latency-critical path on which cudaMalloc is not allowed.
+ * It computes exactly what rocs_lcb_forward computes, with the same kernel, but keeps its
+ * scratch (status word, ready flags, fp32 Z) in a fixed array of
+ * ROCS_LCB_NOALLOC_SCRATCH_BYTES bytes of device memory that the library declares; it
+ * allocates and frees nothing.  args->workspace and args->workspace_bytes are ignored.
+ *   - Sizes whose scratch (rocs_lcb_workspace_size(args)) exceeds the array are rejected
+ *     with ROCS_ERR_WORKSPACE (with o_c = d = 128 that is about 127 requests).
+ *   - Every GPU that loads the library holds the array until the process exits.
+ *   - All calls on a device share the array: calls that can overlap on the GPU race and
+ *     must be serialised by the caller.  The array keeps the last call's contents; each
+ *     call clears the status word and flags itself.
+ *   - The first call on a device looks up the array's device address (once per device);
+ *     make that first call before any stream capture starts.
+ *   - Device-side status is kept in the array's own header and is not readable through
+ *     rocs_read_status(); host-side validation errors are returned as for rocs_lcb_forward. */
+#define ROCS_LCB_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+ROCS_API int rocs_lcb_forward_noalloc(const rocs_lcb_args* args, rocs_stream_t stream);
+
 /* ------------------------------------------------------------------------------------
  * IKBO-DCA  (section 3.2 Eq. (13); section 4.3)
  *
