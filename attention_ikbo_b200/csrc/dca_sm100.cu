@@ -22,7 +22,10 @@
 //     accumulating in TMEM.  The issuer alternates [PV_A, S_A] and [PV_B, S_B] so the
 //     tensor core works on one tile while the softmax warps of the other tile run.
 //   * online softmax in the exp2 domain with lazy rescaling: O and the running sum are
-//     rescaled only when a row's maximum grows by more than 2^8.
+//     rescaled only when a row's maximum grows by more than 2^8; row maxima with 3-input max
+//     chains, exponent arguments and row sums with packed fp32x2 FMA/ADD, exp2 on the MUFU.
+//   * three warpgroups (producer/issuer, tile A softmax, tile B softmax); setmaxnreg moves
+//     registers from the first to the other two so all 128 scores of a row stay in registers.
 //   * work units are claimed from a global ticket in a table ordered longest request first
 //     (load balance), units of one (request, head) adjacent (K/V L2 locality; section 4.3.1's
 //     grid reordering, expressed as the claim order of a persistent kernel).
@@ -35,7 +38,13 @@ namespace {
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
-constexpr int kSoftmaxWarp0 = 4;  // warps 4..7 tile A, 8..11 tile B
+constexpr int kSoftmaxWarp0 = 4;  // warpgroup 1 (warps 4..7) tile A, warpgroup 2 (8..11) tile B
+// Register split (setmaxnreg): launched at kLaunchRegs per thread (checked on the host before
+// the first launch), warpgroup 0 gives registers back, the two softmax warpgroups take them:
+//   4 warps x 32 x kRegsCtl + 8 warps x 32 x kRegsSoftmax == 384 x kLaunchRegs,
+// and per SM sub-partition (warps w, w+4, w+8) kRegsCtl + 2 kRegsSoftmax == 3 kLaunchRegs.
+constexpr uint32_t kLaunchRegs = 168, kRegsCtl = 120, kRegsSoftmax = 192;
+static_assert(4 * 32 * kRegsCtl + 8 * 32 * kRegsSoftmax == kThreads * kLaunchRegs, "register split");
 constexpr int BM = 128, BN = 128;
 constexpr int kRowsPerUnit = 2 * BM;
 
@@ -150,7 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
   const uint32_t tmem_base = *s_tmem;
   // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+DH) O_B [256+DH,256+2DH); P_X over S_X [0,64)
 
-  if (warp == kProducerWarp) {
+  if (warp < kSoftmaxWarp0) {
+   // warpgroup 0: hand registers to the softmax warpgroups, then producer / issuer / idle
+   reg_dealloc<kRegsCtl>();
+   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -203,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
           mbar_drain(&ring_full[k % kRing], (k / kRing) & 1, 20000000ull);
       }
     }
-  } else if (warp == kMmaWarp) {
+   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);  // S = Q K^T : both K-major
@@ -225,18 +237,19 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         if (++rs == kRing) { rs = 0; rph ^= 1; }
       };
       auto issue_s = [&](int x, uint32_t kslot) {
-        const uint32_t qa = q0 + x * L::kTile;
+        const uint64_t ad = sdesc_sw128(q0 + x * L::kTile, 16, 1024), bd = sdesc_sw128(kslot, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk)
-          umma_ss(tmem_base + x * 128, sdesc_sw128(qa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024),
-                  sdesc_sw128(kslot + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024), idesc_s, kk != 0);
+          umma_ss(tmem_base + x * 128, sdesc_add(ad, (kk >> 2) * (BM * 128) + (kk & 3) * 32),
+                  sdesc_add(bd, (kk >> 2) * (BN * 128) + (kk & 3) * 32), idesc_s, kk != 0);
         umma_commit(&s_full[x]);
       };
       auto issue_pv = [&](int x, uint32_t vslot, bool acc) {
+        const uint64_t vd = sdesc_sw128(vslot, BN * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(tmem_base + 256 + x * DH, tmem_base + x * 128 + kk * 8,
-                  sdesc_sw128(vslot + kk * 2048, BN * 128, 1024), idesc_o, (acc || kk != 0) ? 1u : 0u);
+          umma_ts(tmem_base + 256 + x * DH, tmem_base + x * 128 + kk * 8, sdesc_add(vd, kk * 2048), idesc_o,
+                  (acc || kk != 0) ? 1u : 0u);
       };
       auto wait_p = [&](int x, bool first_pv) -> bool {
         if (!mbar_wait(&p_full[x], pph[x], ctl, 601)) return false;
@@ -299,8 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       umma_commit(drain_bar);
       mbar_drain(drain_bar, 0, 50000000ull);
     }
-  } else if (warp >= kSoftmaxWarp0) {
+   }
+  } else {
     // ------------------------------------------------------------------ softmax + epilogue
+    reg_alloc<kRegsSoftmax>();
     const int x = (warp - kSoftmaxWarp0) >> 2;  // 0: tile A, 1: tile B
     const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
     const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
@@ -346,11 +361,18 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
             for (int k = 0; k < 32; ++k)
               if (c4 * 32 + k >= kvalid) sv[c4][k] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        float mq[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mq[k] = -INFINITY;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
 #pragma unroll
-          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, __uint_as_float(sv[c4][k]));
+          for (int k = 0; k < 16; ++k) {
+            float y;
+            asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(mq[k & 7]), "f"(__uint_as_float(sv[c4][2 * k])), "f"(__uint_as_float(sv[c4][2 * k + 1])));
+            mq[k & 7] = y;
+          }
+        const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
         const float mxs = mx * c;
         if (j == 0) {
           m_used = mxs;
@@ -369,20 +391,31 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
           }
           m_used = m_new;
         }
-        const float nm = -m_used;
-        float lsum = 0.f;
+        uint64_t c2, nm2, ls0 = 0, ls1 = 0;
+        asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(c));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(nm2) : "f"(-m_used));
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const float p0 = ex2(fmaf(__uint_as_float(sv[c4][2 * k]), c, nm));
-            const float p1 = ex2(fmaf(__uint_as_float(sv[c4][2 * k + 1]), c, nm));
-            lsum += p0 + p1;
+            uint64_t sp, xp, ep;
+            asm("mov.b64 %0, {%1, %2};" : "=l"(sp) : "r"(sv[c4][2 * k]), "r"(sv[c4][2 * k + 1]));
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(xp) : "l"(sp), "l"(c2), "l"(nm2));
+            float x0, x1;
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(xp));
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            asm("mov.b64 %0, {%1, %2};" : "=l"(ep) : "f"(p0), "f"(p1));
+            if (k & 1) asm("add.f32x2 %0, %1, %2;" : "=l"(ls1) : "l"(ls1), "l"(ep));
+            else asm("add.f32x2 %0, %1, %2;" : "=l"(ls0) : "l"(ls0), "l"(ep));
             pk[k] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(s_addr + c4 * 16, pk);  // P (bf16 pairs) over the first 64 columns of S
+          tmem_st16(s_addr + c4 * 16, pk);
         }
+        float la, lb, lc, ld;
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(la), "=f"(lb) : "l"(ls0));
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(lc), "=f"(ld) : "l"(ls1));
+        const float lsum = (la + lb) + (lc + ld);
         l += lsum;
         tmem_st_wait();
         tc_fence_before();
@@ -498,6 +531,9 @@ static cudaError_t launch_t(const DcaParams& p, int grid, cudaStream_t st) {
   auto k = rocs_dca_sm100_kernel<DH>;
   static bool attr_set = false;
   if (!attr_set) {
+    // the setmaxnreg split is only valid for the register count it was computed for
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, k) != cudaSuccess || fa.numRegs != (int)kLaunchRegs) return cudaErrorInvalidConfiguration;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::alloc_bytes);
     if (e != cudaSuccess) return e;
     attr_set = true;

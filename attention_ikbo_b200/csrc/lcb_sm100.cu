@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&p.tm_xc);
+      if (cbeg < cend) tma_prefetch_desc(&p.tm_xc);
       tma_prefetch_desc(&p.tm_xr);
       int n_issued = 0;
       bool ok = true;
@@ -183,11 +183,11 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
         for (int kb = 0; kb < kblocks && ok; ++kb) {
           if (!mbar_wait(&full[s], ph, ctl, 203)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(s_ring + s * kSlot), b0 = a0 + 16384;
+          const uint32_t a0 = smem_u32(s_ring + s * kSlot);
+          const uint64_t ad = sdesc_sw128(a0, 16, 1024), bd = sdesc_sw128(a0 + 16384, 8192, 1024);
 #pragma unroll
           for (int kin = 0; kin < 4; ++kin)
-            umma_ss(d_tmem, sdesc_sw128(a0 + kin * 32, 16, 1024), sdesc_sw128(b0 + kin * 2048, 8192, 1024), idesc,
-                    (kb | kin) != 0);
+            umma_ss(d_tmem, sdesc_add(ad, kin * 32), sdesc_add(bd, kin * 2048), idesc, (kb | kin) != 0);
           umma_commit(&empty[s]);
           if (++s == kStages) { s = 0; ph ^= 1; }
         }
@@ -196,17 +196,16 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
         if (++ab == 2) { ab = 0; aph ^= 1; }
       }
       if (ok && cbeg < cend && !mbar_wait(wcc_bar, 0, ctl, 204)) ok = false;
-      const uint32_t wcc0 = smem_u32(s_wcc);
+      const uint64_t wccd = sdesc_sw128(smem_u32(s_wcc), 16, 1024);
       for (int i = cbeg; ok && i < cend; ++i) {  // candidate tiles
         if (!mbar_wait(&acc_empty[ab], aph ^ 1, ctl, 205)) { ok = false; break; }
         if (!mbar_wait(&full[s], ph, ctl, 206)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * D;
-        const uint32_t b0 = smem_u32(s_ring + s * kSlot);
+        const uint64_t bd = sdesc_sw128(smem_u32(s_ring + s * kSlot), NC * 128, 1024);
 #pragma unroll
         for (int ks = 0; ks < NC / 16; ++ks)
-          umma_ss(d_tmem, sdesc_sw128(wcc0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                  sdesc_sw128(b0 + ks * 2048, NC * 128, 1024), idesc, ks != 0);
+          umma_ss(d_tmem, sdesc_add(wccd, (ks >> 2) * 16384 + (ks & 3) * 32), sdesc_add(bd, ks * 2048), idesc, ks != 0);
         umma_commit(&empty[s]);
         umma_commit(&acc_full[ab]);
         if (++s == kStages) { s = 0; ph ^= 1; }

@@ -98,11 +98,11 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_proj_sm100_kernel(const __gr
         for (int kb = 0; kb < kb_n; ++kb) {
           if (!mbar_wait(&full[s], ph, ctl, 903)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + s * kStage), b0 = a0 + kA;
+          const uint32_t a0 = smem_u32(smem + s * kStage);
+          const uint64_t ad = sdesc_sw128(a0, 16, 1024), bd = sdesc_sw128(a0 + kA, 16, 1024);
 #pragma unroll
           for (int kin = 0; kin < BK / 16; ++kin)
-            umma_ss(d, sdesc_sw128(a0 + kin * 32, 16, 1024), sdesc_sw128(b0 + kin * 32, 16, 1024), idesc,
-                    (kb | kin) != 0);
+            umma_ss(d, sdesc_add(ad, kin * 32), sdesc_add(bd, kin * 32), idesc, (kb | kin) != 0);
           umma_commit(&empty[s]);
           if (++s == kStages) { s = 0; ph ^= 1; }
         }
