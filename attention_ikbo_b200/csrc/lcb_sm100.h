@@ -7,7 +7,7 @@ namespace rocs {
 // Persistent IKBO-LCB kernel (bf16 in, fp32 accumulate, bf16 out).
 struct LcbParams {
   CUtensorMap tm_xc;   // X^C  viewed as [C*n_c, d],  box {64, n_c}
-  CUtensorMap tm_xr;   // X^R  viewed as [R*n_r, d],  box {64, 128}
+  CUtensorMap tm_xr;   // X^R  viewed as [R*n_r, d],  box {64, 64}
   CUtensorMap tm_wcc;  // W_CC [o_c, n_c],            box {64, 128}
   CUtensorMap tm_wrr;  // W_RR [o_r, n_r],            box {64, 128}
   CUtensorMap tm_wcr;  // W_CR [o_c, n_r],            box {64, 128}
