@@ -26,6 +26,7 @@ from ._binding import (  # noqa: F401
     rocs_dca_forward_expand,
     rocs_lcb_forward,
     rocs_lcb_forward_expand,
+    rocs_lcb_forward_fault_injection,
     rocs_lcb_forward_noalloc,
     rocs_proj_forward,
     rocs_read_status,

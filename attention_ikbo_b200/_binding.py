@@ -64,6 +64,7 @@ def load_library():
             getattr(lib, name).argtypes = argt
         for name, argt in [("rocs_lcb_forward", [P(LcbArgs), _vp]), ("rocs_lcb_forward_expand", [P(LcbArgs), _vp]),
                            ("rocs_lcb_forward_noalloc", [P(LcbArgs), _vp]),
+                           ("rocs_lcb_forward_fault_injection", [P(LcbArgs), _vp, _i64, _i64]),
                            ("rocs_dca_forward", [P(DcaArgs), _vp]), ("rocs_proj_forward", [P(ProjArgs), _vp]),
                            ("rocs_dca_forward_expand", [P(DcaArgs), _i64, _vp]),
                            ("rocs_read_status", [_vp, _vp, P(_i32), P(_i32)])]:
@@ -178,6 +179,19 @@ def rocs_lcb_forward_noalloc(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y
     a, keep, y_req, y_cand = _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y_cand)
     _check(lib.rocs_lcb_forward_noalloc(ctypes.byref(a), _stream(stream)), "rocs_lcb_forward_noalloc")
     return y_req, y_cand
+
+
+def rocs_lcb_forward_fault_injection(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, skip_release_request,
+                                     wait_limit_ns, stream=None):
+    """Test hook: LCB whose request ``skip_release_request`` never signals its Z; the kernel must end
+    with ROCS_ERR_TIMEOUT after ``wait_limit_ns``.  Returns the workspace (read it with rocs_read_status)."""
+    lib = load_library()
+    a, keep, y_req, y_cand = _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, None, None)
+    ws = _workspace(lib.rocs_lcb_workspace_size(ctypes.byref(a)), x_req.device, None)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check(lib.rocs_lcb_forward_fault_injection(ctypes.byref(a), _stream(stream), int(skip_release_request),
+                                                int(wait_limit_ns)), "rocs_lcb_forward_fault_injection")
+    return ws
 
 
 def rocs_lcb_forward_expand(*args, **kw):

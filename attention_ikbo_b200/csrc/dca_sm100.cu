@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
-  const Ctl ctl{s_abort, p.ws};
+  const Ctl ctl{s_abort, p.ws, (unsigned long long)p.wait_limit_ns};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRing; ++s) {

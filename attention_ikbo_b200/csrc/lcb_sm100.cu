@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
-  const Ctl ctl{s_abort, p.ws};
+  const Ctl ctl{s_abort, p.ws, (unsigned long long)p.wait_limit_ns};
 
   const int R = p.R, C = p.C;
   const int mt_r = p.o_r / OC;                // 128-row slices of Y^R per request
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
         if (lane == 0) {
           mbar_arrive(&acc_empty[ab]);
           __threadfence();
-          red_release_gpu_add(&p.flags[r], 1);  // 4 warps x 1 = this request's Z is complete
+          if (r != p.skip_release) red_release_gpu_add(&p.flags[r], 1);  // 4 warps x 1 = this request's Z is complete
         }
       } else {
         const int u = item - R, r = u / mt_r, mt = u % mt_r;

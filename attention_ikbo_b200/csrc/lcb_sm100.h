@@ -18,6 +18,8 @@ struct LcbParams {
   int* flags;               // [R], incremented by each epilogue warp of the Z tile
   WsHeader* ws;
   int R, C, n_r, o_r;
+  long long wait_limit_ns;  // limit of every wait in the kernel
+  int skip_release;         // fault injection: the Z tile of this request never releases its flag (-1: none)
 };
 cudaError_t launch_lcb_sm100(const LcbParams& p, int d, int n_c, int grid, cudaStream_t st);
 
@@ -44,6 +46,7 @@ struct DcaParams {
   WsHeader* ws;
   int R, q, H, n_units;
   float scale_log2;  // softmax scale * log2(e)
+  long long wait_limit_ns;
 };
 cudaError_t launch_dca_sm100(const DcaParams& p, int dh, int grid, cudaStream_t st);
 
@@ -64,6 +67,7 @@ struct ProjParams {
   __nv_bfloat16* out;  // [M, N]
   WsHeader* ws;
   int M, N, K;
+  long long wait_limit_ns;
 };
 cudaError_t launch_proj_sm100(const ProjParams& p, int grid, cudaStream_t st);
 

@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_proj_sm100_kernel(const __gr
 
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = threadIdx.x & 31;
-  const Ctl ctl{s_abort, p.ws};
+  const Ctl ctl{s_abort, p.ws, (unsigned long long)p.wait_limit_ns};
   const int mt = (p.M + BM - 1) / BM, nt = p.N / BN, tiles = mt * nt, kb_n = p.K / BK;
 
   if (threadIdx.x == 0) {

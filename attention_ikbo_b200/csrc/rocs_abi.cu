@@ -111,7 +111,13 @@ int lcb_validate(const rocs_lcb_args* a, int64_t* C) {
   return ROCS_OK;
 }
 
-int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaStream_t st, int* launches) {
+struct LcbOpts {
+  long long wait_ns = kDefaultWaitLimitNs;
+  int skip_release = -1;  // fault injection only
+};
+
+int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaStream_t st, int* launches,
+            const LcbOpts& opts = LcbOpts()) {
   const LcbLayout L = lcb_body(a->R, a->o_c, a->d);
   if (w == reinterpret_cast<uint8_t*>(hdr + 1)) {
     if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader) + (size_t)a->R * sizeof(int), st) != cudaSuccess) return ROCS_ERR_CUDA;
@@ -165,6 +171,8 @@ int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaSt
   p.C = (int)C;
   p.n_r = (int)a->n_r;
   p.o_r = (int)a->o_r;
+  p.wait_limit_ns = opts.wait_ns;
+  p.skip_release = opts.skip_release;
   const int64_t n_req_tiles = a->R * (1 + a->o_r / 128);
   int64_t grid = C > n_req_tiles ? C : n_req_tiles;
   if (grid > sm_count()) grid = sm_count();
@@ -258,6 +266,7 @@ int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHea
   p.H = (int)a->H;
   p.n_units = (int)n_units;
   p.scale_log2 = a->scale * 1.4426950408889634f;
+  p.wait_limit_ns = kDefaultWaitLimitNs;
   int64_t grid = n_units < sm_count() ? n_units : sm_count();
   if (launch_dca_sm100(p, (int)a->dh, (int)grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
   *launches = 2;
@@ -298,6 +307,26 @@ int rocs_lcb_forward(const rocs_lcb_args* a, rocs_stream_t stream) {
   int launches = 0;
   WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
   rc = lcb_run(a, C, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream), &launches);
+  if (rc == ROCS_OK) g_last_launches = launches;
+  return rc;
+}
+
+int rocs_lcb_forward_fault_injection(const rocs_lcb_args* a, rocs_stream_t stream, int64_t skip_release_request,
+                                     int64_t wait_limit_ns) {
+  int64_t C = 0;
+  int rc = lcb_validate(a, &C);
+  if (rc) return rc;
+  if (a->dtype != ROCS_BF16) return ROCS_ERR_UNSUPPORTED;  // the ready flags exist in the bf16 kernel only
+  if (skip_release_request < -1 || skip_release_request >= a->R) return ROCS_ERR_INVALID_ARG;
+  if (wait_limit_ns < 1000000 || wait_limit_ns > 10000000000ll) return ROCS_ERR_INVALID_ARG;
+  if (!a->workspace || a->workspace_bytes < lcb_bytes(a) || (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ROCS_ERR_WORKSPACE;
+  LcbOpts o;
+  o.wait_ns = wait_limit_ns;
+  o.skip_release = (int)skip_release_request;
+  int launches = 0;
+  WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
+  rc = lcb_run(a, C, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream), &launches, o);
   if (rc == ROCS_OK) g_last_launches = launches;
   return rc;
 }
@@ -354,6 +383,7 @@ int rocs_proj_forward(const rocs_proj_args* a, rocs_stream_t stream) {
   p.M = (int)a->M;
   p.N = (int)a->N;
   p.K = (int)a->K;
+  p.wait_limit_ns = kDefaultWaitLimitNs;
   const int64_t tiles = ((a->M + 127) / 128) * (a->N / 256);
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   if (launch_proj_sm100(p, grid, st) != cudaSuccess) return ROCS_ERR_CUDA;

@@ -28,9 +28,9 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
-#ifndef ROCS_WAIT_LIMIT_NS
-#define ROCS_WAIT_LIMIT_NS 2000000000ull  // 2 s: far above any legitimate wait here
-#endif
+// Default limit of every wait (kernels receive it as a launch parameter): far above any
+// legitimate wait in these kernels, short enough that a broken hand-off ends as an error.
+constexpr long long kDefaultWaitLimitNs = 2000000000ll;  // 2 s
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -43,10 +43,11 @@ __device__ __forceinline__ void record_error(WsHeader* ws, int code, int detail)
   if (atomicCAS(&ws->code, 0, code) == 0) atomicExch(&ws->detail, detail);
 }
 
-// Per-CTA control block: shared abort flag + global status.
+// Per-CTA control block: shared abort flag + global status + wait limit.
 struct Ctl {
   volatile int* abort;  // shared memory
   WsHeader* ws;
+  unsigned long long limit_ns;
   __device__ __forceinline__ bool aborted() const { return *abort != 0; }
   __device__ __forceinline__ void fail(int code, int detail) const {
     *abort = 1;
@@ -88,7 +89,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (ctl.aborted()) return false;
-      if (globaltimer() - t0 > ROCS_WAIT_LIMIT_NS) {
+      if (globaltimer() - t0 > ctl.limit_ns) {
         ctl.fail(ROCS_ERR_TIMEOUT, where);
         return false;
       }
@@ -121,7 +122,7 @@ __device__ __forceinline__ bool wait_flag_geq(const int* flag, int target, const
     __nanosleep(64);
     if ((it & 15u) == 0) {
       if (ctl.aborted()) return false;
-      if (globaltimer() - t0 > ROCS_WAIT_LIMIT_NS) {
+      if (globaltimer() - t0 > ctl.limit_ns) {
         ctl.fail(ROCS_ERR_TIMEOUT, where);
         return false;
       }

@@ -121,6 +121,16 @@ ROCS_API int rocs_lcb_forward(const rocs_lcb_args* args, rocs_stream_t stream);
 ROCS_API size_t rocs_lcb_expand_workspace_size(const rocs_lcb_args* args);
 ROCS_API int rocs_lcb_forward_expand(const rocs_lcb_args* args, rocs_stream_t stream);
 
+/* Fault-injection hook for testing the bounded waits (not for production use; the paper has
+ * no counterpart).  Identical to rocs_lcb_forward with dtype ROCS_BF16, except that the request
+ * tile computing Z for request `skip_release_request` (-1: none) never releases its ready flag, so
+ * every candidate epilogue of that request waits until `wait_limit_ns` (1e6 .. 1e10) expires.  The
+ * kernel then finishes with ROCS_ERR_TIMEOUT in the workspace status word (read it with
+ * rocs_read_status): no trap, no hang, and the CUDA context stays usable.  Outputs of the
+ * affected request are undefined.  ROCS_ERR_UNSUPPORTED for ROCS_F32. */
+ROCS_API int rocs_lcb_forward_fault_injection(const rocs_lcb_args* args, rocs_stream_t stream,
+                                              int64_t skip_release_request, int64_t wait_limit_ns);
+
 /* IKBO-LCB without a caller workspace.  The paper has no counterpart: this entry point
  * exists for callers that cannot hand the library device memory -- e.g. a plugin inside a
  * serving process whose device memory is fully reserved by the host framework's own pool

@@ -31,7 +31,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_symbols()
-    assert len(names) >= 13
+    assert len(names) >= 15
     for n in names:
         assert hasattr(lib, n), n
 
@@ -108,3 +108,13 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(b, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         b.load_library()
+
+
+def test_fault_injection_host_validation(lib):
+    import attention_ikbo_b200 as m
+
+    a, keep = _lcb_args(m, [0, 3, 6], ws_bytes=1 << 20)
+    assert lib.rocs_lcb_forward_fault_injection(ctypes.byref(a), None, 5, 10_000_000) == 1  # no request 5
+    assert lib.rocs_lcb_forward_fault_injection(ctypes.byref(a), None, 0, 10) == 1  # limit below 1 ms
+    f32, keep2 = _lcb_args(m, [0, 3, 6], dtype=0, ws_bytes=1 << 20)
+    assert lib.rocs_lcb_forward_fault_injection(ctypes.byref(f32), None, 0, 10_000_000) == 3
