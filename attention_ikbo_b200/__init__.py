@@ -11,6 +11,8 @@ Operations ("ROCS: Request-Oriented Compute Sharing ...", arXiv:2607.27744):
     decomposition, broadcast-add fused into the candidate GEMM epilogue (section 4.2).
   * :func:`rocs_dca_forward` -- section 3.2 Eq. (13) candidate cross attention over K/V
     stored once per request (section 4.3).
+  * :func:`rocs_dca_block_forward` -- both query groups of Eq. (13) with the K/V projections
+    done once per request (section 4.1).
   * :func:`rocs_proj_forward` -- linear query projection of the chained block (Eq. 12).
 """
 from ._binding import (  # noqa: F401
@@ -22,6 +24,7 @@ from ._binding import (  # noqa: F401
     lib_path,
     load_library,
     offsets,
+    rocs_dca_block_forward,
     rocs_dca_forward,
     rocs_dca_forward_expand,
     rocs_lcb_forward,

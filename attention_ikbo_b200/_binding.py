@@ -34,7 +34,15 @@ class DcaArgs(ctypes.Structure):
     _fields_ = [("R", _i64), ("q", _i64), ("H", _i64), ("dh", _i64), ("scale", _f32),
                 ("cand_off_dev", _vp), ("cand_off_host", _vp), ("seq_off_dev", _vp), ("seq_off_host", _vp),
                 ("q_ptr", _vp), ("k_ptr", _vp), ("v_ptr", _vp), ("o_ptr", _vp), ("lse_ptr", _vp),
-                ("workspace", _vp), ("workspace_bytes", _sz)]
+                ("workspace", _vp), ("workspace_bytes", _sz), ("kv_ld", _i64)]
+
+
+class DcaBlockArgs(ctypes.Structure):
+    _fields_ = [("R", _i64), ("q", _i64), ("q_req", _i64), ("H", _i64), ("dh", _i64), ("d_s", _i64),
+                ("scale", _f32), ("cand_off_dev", _vp), ("cand_off_host", _vp), ("seq_off_dev", _vp),
+                ("seq_off_host", _vp), ("s_seq", _vp), ("w_kv", _vp), ("q_c", _vp), ("q_r", _vp),
+                ("o_c", _vp), ("lse_c", _vp), ("o_r", _vp), ("lse_r", _vp), ("workspace", _vp),
+                ("workspace_bytes", _sz)]
 
 
 class ProjArgs(ctypes.Structure):
@@ -59,7 +67,8 @@ def load_library():
         P = ctypes.POINTER
         for name, argt in [("rocs_lcb_workspace_size", [P(LcbArgs)]), ("rocs_lcb_expand_workspace_size", [P(LcbArgs)]),
                            ("rocs_dca_workspace_size", [P(DcaArgs)]), ("rocs_proj_workspace_size", [P(ProjArgs)]),
-                           ("rocs_dca_expand_workspace_size", [P(DcaArgs), _i64])]:
+                           ("rocs_dca_expand_workspace_size", [P(DcaArgs), _i64]),
+                           ("rocs_dca_block_workspace_size", [P(DcaBlockArgs)])]:
             getattr(lib, name).restype = _sz
             getattr(lib, name).argtypes = argt
         for name, argt in [("rocs_lcb_forward", [P(LcbArgs), _vp]), ("rocs_lcb_forward_expand", [P(LcbArgs), _vp]),
@@ -67,6 +76,7 @@ def load_library():
                            ("rocs_lcb_forward_fault_injection", [P(LcbArgs), _vp, _i64, _i64]),
                            ("rocs_dca_forward", [P(DcaArgs), _vp]), ("rocs_proj_forward", [P(ProjArgs), _vp]),
                            ("rocs_dca_forward_expand", [P(DcaArgs), _i64, _vp]),
+                           ("rocs_dca_block_forward", [P(DcaBlockArgs), _vp]),
                            ("rocs_read_status", [_vp, _vp, P(_i32), P(_i32)])]:
             getattr(lib, name).restype = ctypes.c_int
             getattr(lib, name).argtypes = argt
@@ -249,6 +259,41 @@ def rocs_dca_forward(q_t, k_t, v_t, cand_off, seq_off, q_tokens, scale, o=None, 
 
 def rocs_dca_forward_expand(*args, expand_chunk=1024, **kw):
     return rocs_dca_forward(*args, expand_chunk=expand_chunk, **kw)
+
+
+def rocs_dca_block_forward(s_seq, w_kv, q_c, q_r, cand_off, seq_off, q_tokens, q_req_tokens, scale, o_c=None,
+                           o_r=None, lse=True, workspace=None, stream=None):
+    """DCA block (both query groups of Eq. 13): K/V projected once per request with the stacked
+    weights ``w_kv = [W_K^C; W_V^C; W_K^R; W_V^R]``, then IKBO-DCA for the candidates and attention of
+    every request's own ``q_req_tokens`` queries.  Returns ``(o_c, lse_c, o_r, lse_r)``."""
+    lib = load_library()
+    dev = q_c.device
+    co_d, co_h = _offsets(cand_off, dev)
+    so_d, so_h = _offsets(seq_off, dev)
+    R = len(co_h) - 1
+    H, dh = q_c.shape[1], q_c.shape[2]
+    o_c = torch.empty(q_c.shape, dtype=torch.bfloat16, device=dev) if o_c is None else o_c
+    o_r = torch.empty(q_r.shape, dtype=torch.bfloat16, device=dev) if o_r is None else o_r
+    lse_c = torch.empty(q_c.shape[:2], dtype=torch.float32, device=dev) if lse else None
+    lse_r = torch.empty(q_r.shape[:2], dtype=torch.float32, device=dev) if lse else None
+    for t in (s_seq, w_kv, q_c, q_r, o_c, o_r):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16):
+            raise RocsError(1, "DCA block tensors must be contiguous bf16 CUDA tensors")
+    a = DcaBlockArgs(R=R, q=q_tokens, q_req=q_req_tokens, H=H, dh=dh, d_s=s_seq.shape[1], scale=float(scale),
+                     cand_off_dev=co_d.data_ptr(), cand_off_host=co_h.ctypes.data, seq_off_dev=so_d.data_ptr(),
+                     seq_off_host=so_h.ctypes.data, s_seq=s_seq.data_ptr() if s_seq.numel() else None,
+                     w_kv=w_kv.data_ptr(), q_c=q_c.data_ptr() if q_c.numel() else None, q_r=q_r.data_ptr(),
+                     o_c=o_c.data_ptr() if o_c.numel() else None, o_r=o_r.data_ptr(),
+                     lse_c=lse_c.data_ptr() if lse_c is not None and lse_c.numel() else None,
+                     lse_r=lse_r.data_ptr() if lse_r is not None else None)
+    nbytes = lib.rocs_dca_block_workspace_size(ctypes.byref(a))
+    if nbytes == 0:
+        _check(lib.rocs_dca_block_forward(ctypes.byref(a), _stream(stream)), "rocs_dca_block_forward")
+    ws = _workspace(nbytes, dev, workspace)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check(lib.rocs_dca_block_forward(ctypes.byref(a), _stream(stream)), "rocs_dca_block_forward")
+    rocs_dca_block_forward.last_workspace = ws
+    return o_c, lse_c, o_r, lse_r
 
 
 def rocs_proj_forward(inp, w, out=None, workspace=None, stream=None):

@@ -83,6 +83,11 @@ __global__ void rocs_expand_kv_kernel(const uint4* k, const uint4* v, uint4* k_o
   }
 }
 
+cudaError_t launch_ident(int32_t* out, int n, cudaStream_t st) {  // out[k] = k, k = 0..n
+  rocs_expand_ident_kernel<<<(n + 256) / 256 < 4096 ? (n + 256) / 256 : 4096, 256, 0, st>>>(out, n, n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_expand_rows(const void* src, void* dst, const int32_t* cand_off, int R, int C, int64_t row_bytes,
                                int64_t rows_per_item, cudaStream_t st) {
   const int64_t item_vec = row_bytes * rows_per_item / 16;
@@ -213,6 +218,7 @@ int rocs_dca_forward_expand(const rocs_dca_args* a, int64_t chunk, rocs_stream_t
   if (chunk <= 0 || chunk > (1 << 20)) return ROCS_ERR_INVALID_ARG;
   int rc = dca_validate_ext(a, &C, &T);
   if (rc) return rc;
+  if (a->kv_ld != 0 && a->kv_ld != a->H * a->dh) return ROCS_ERR_UNSUPPORTED;  // the copies assume dense rows
   const DcaExpandLayout L = dca_expand_layout(a, C, chunk);
   if (!a->workspace || a->workspace_bytes < L.bytes || (reinterpret_cast<uintptr_t>(a->workspace) & 255))
     return ROCS_ERR_WORKSPACE;

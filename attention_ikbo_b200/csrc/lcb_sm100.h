@@ -71,6 +71,9 @@ struct ProjParams {
 };
 cudaError_t launch_proj_sm100(const ProjParams& p, int grid, cudaStream_t st);
 
+// out[k] = k for k = 0..n (the identity candidate map: every request its own single candidate).
+cudaError_t launch_ident(int32_t* out, int n, cudaStream_t st);
+
 // Explicit-expand baseline helpers.
 cudaError_t launch_expand_rows(const void* src, void* dst, const int32_t* cand_off, int R, int C, int64_t row_bytes,
                                int64_t rows_per_item, cudaStream_t st);

@@ -220,16 +220,17 @@ int dca_validate(const rocs_dca_args* a, int64_t* C, int64_t* T) {
   for (const void* p : ptrs)
     if (p && !al16(p)) return ROCS_ERR_INVALID_ARG;
   if (a->lse_ptr && (reinterpret_cast<uintptr_t>(a->lse_ptr) & 3u)) return ROCS_ERR_INVALID_ARG;
+  if (a->kv_ld != 0 && (a->kv_ld < a->H * a->dh || (a->kv_ld * 2) % 16)) return ROCS_ERR_UNSUPPORTED;
   if (*C * a->q >= (int64_t(1) << 31) || *T >= (int64_t(1) << 31) || a->H * a->dh >= (int64_t(1) << 20))
     return ROCS_ERR_UNSUPPORTED;
   return ROCS_OK;
 }
 
 int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHeader* hdr, uint8_t* w,
-            cudaStream_t st, int* launches) {
+            cudaStream_t st, int* launches, bool reset_header = true) {
   const DcaLayout L = dca_body(a->R, n_units);
   if (n_units >= (int64_t(1) << 31)) return ROCS_ERR_UNSUPPORTED;
-  if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return ROCS_ERR_CUDA;
+  if (reset_header && cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return ROCS_ERR_CUDA;
   if (n_units == 0) return ROCS_OK;
   DcaSchedParams sp;
   sp.cand_off = a->cand_off_dev;
@@ -245,11 +246,11 @@ int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHea
   if (launch_dca_schedule(sp, st) != cudaSuccess) return ROCS_ERR_CUDA;
   DcaParams p;
   std::memset(&p, 0, sizeof(p));
-  const uint64_t hd = a->H * a->dh, rb = hd * 2;
+  const uint64_t hd = a->H * a->dh, rb = hd * 2, kvb = (a->kv_ld ? a->kv_ld : hd) * 2;
   bool ok = tmap_bf16(&p.tm_q, a->q_ptr, hd, (uint64_t)C * a->q, rb, 64, 128);
   if (T > 0) {
-    ok &= tmap_bf16(&p.tm_k, a->k_ptr, hd, (uint64_t)T, rb, 64, 128);
-    ok &= tmap_bf16(&p.tm_v, a->v_ptr, hd, (uint64_t)T, rb, 64, 128);
+    ok &= tmap_bf16(&p.tm_k, a->k_ptr, hd, (uint64_t)T, kvb, 64, 128);
+    ok &= tmap_bf16(&p.tm_v, a->v_ptr, hd, (uint64_t)T, kvb, 64, 128);
   } else {  // never loaded (every request has zero keys); any valid descriptor will do
     p.tm_k = p.tm_q;
     p.tm_v = p.tm_q;
@@ -351,6 +352,117 @@ int rocs_dca_forward(const rocs_dca_args* a, rocs_stream_t stream) {
                &launches);
   if (rc == ROCS_OK) g_last_launches = launches;
   return rc;
+}
+
+// ---- DCA block: projection GEMM + candidate-group and request-group attention
+namespace {
+struct BlockLayout {
+  size_t ident, kv, body_c, body_r, bytes;
+  int64_t C, T, units_c, units_r;
+};
+int block_layout(const rocs_dca_block_args* a, BlockLayout* L) {
+  if (!a || a->R < 0 || a->q <= 0 || a->q_req <= 0 || a->H <= 0 || a->d_s <= 0) return ROCS_ERR_INVALID_ARG;
+  if ((a->dh != 64 && a->dh != 128) || a->d_s % 64) return ROCS_ERR_UNSUPPORTED;
+  int rc = check_csr(a->cand_off_host, a->R, &L->C);
+  if (rc) return rc;
+  rc = check_csr(a->seq_off_host, a->R, &L->T);
+  if (rc) return rc;
+  const int64_t hd = a->H * a->dh, rpu = dca_rows_per_unit();
+  if (L->T * 4 * hd >= (int64_t(1) << 31) || L->C * a->q >= (int64_t(1) << 31)) return ROCS_ERR_UNSUPPORTED;
+  L->units_c = 0;
+  for (int64_t r = 0; r < a->R; ++r)
+    L->units_c += a->H * ((a->q * (int64_t)(a->cand_off_host[r + 1] - a->cand_off_host[r]) + rpu - 1) / rpu);
+  L->units_r = a->R * a->H * ((a->q_req + rpu - 1) / rpu);
+  L->ident = sizeof(WsHeader);
+  L->kv = a256(L->ident + (size_t)(a->R + 1) * 4);
+  L->body_c = a256(L->kv + (size_t)L->T * 4 * hd * 2);
+  L->body_r = a256(L->body_c + dca_body(a->R, L->units_c).body);
+  L->bytes = L->body_r + dca_body(a->R, L->units_r).body;
+  return ROCS_OK;
+}
+}  // namespace
+
+extern "C" size_t rocs_dca_block_workspace_size(const rocs_dca_block_args* a) {
+  BlockLayout L;
+  return block_layout(a, &L) == ROCS_OK ? L.bytes : 0;
+}
+
+extern "C" int rocs_dca_block_forward(const rocs_dca_block_args* a, rocs_stream_t stream) {
+  BlockLayout L;
+  int rc = block_layout(a, &L);
+  if (rc) return rc;
+  if (!a->workspace || a->workspace_bytes < L.bytes || (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ROCS_ERR_WORKSPACE;
+  const void* ptrs[] = {a->s_seq, a->w_kv, a->q_c, a->q_r, a->o_c, a->o_r};
+  for (const void* p : ptrs)
+    if (p && !al16(p)) return ROCS_ERR_INVALID_ARG;
+  if (a->R > 0 && (!a->cand_off_dev || !a->seq_off_dev || !a->w_kv || !a->q_r || !a->o_r)) return ROCS_ERR_INVALID_ARG;
+  if (L.C > 0 && (!a->q_c || !a->o_c)) return ROCS_ERR_INVALID_ARG;
+  if (L.T > 0 && !a->s_seq) return ROCS_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(a->workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
+  if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return ROCS_ERR_CUDA;
+  if (a->R == 0) return ROCS_OK;
+  int launches = 0;
+  const int64_t hd = a->H * a->dh;
+  uint8_t* kv = w + L.kv;
+  if (L.T > 0) {  // [K^C | V^C | K^R | V^R] = S . W_kv^T, once per request sequence row
+    ProjParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    bool ok = tmap_bf16(&pp.tm_a, a->s_seq, a->d_s, L.T, a->d_s * 2, 64, 128);
+    ok &= tmap_bf16(&pp.tm_b, a->w_kv, a->d_s, 4 * hd, a->d_s * 2, 64, 256);
+    if (!ok) return ROCS_ERR_CUDA;
+    pp.out = reinterpret_cast<__nv_bfloat16*>(kv);
+    pp.ws = hdr;
+    pp.M = (int)L.T;
+    pp.N = (int)(4 * hd);
+    pp.K = (int)a->d_s;
+    pp.wait_limit_ns = kDefaultWaitLimitNs;
+    const int64_t tiles = ((L.T + 127) / 128) * (4 * hd / 256);
+    if (launch_proj_sm100(pp, (int)(tiles < sm_count() ? tiles : sm_count()), st) != cudaSuccess) return ROCS_ERR_CUDA;
+    ++launches;
+  }
+  int32_t* ident = reinterpret_cast<int32_t*>(w + L.ident);
+  if (launch_ident(ident, (int)a->R, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  ++launches;
+  rocs_dca_args d;
+  std::memset(&d, 0, sizeof(d));
+  d.R = a->R;
+  d.H = a->H;
+  d.dh = a->dh;
+  d.scale = a->scale;
+  d.seq_off_dev = a->seq_off_dev;
+  d.seq_off_host = a->seq_off_host;
+  d.kv_ld = 4 * hd;
+  // candidate group (IKBO: K/V at batch B_r, m_i resolved in the kernel)
+  d.q = a->q;
+  d.cand_off_dev = a->cand_off_dev;
+  d.cand_off_host = a->cand_off_host;
+  d.q_ptr = a->q_c;
+  d.k_ptr = kv;
+  d.v_ptr = kv + hd * 2;
+  d.o_ptr = a->o_c;
+  d.lse_ptr = a->lse_c;
+  int n = 0;
+  if (L.C > 0) {
+    rc = dca_run(&d, L.C, L.T, L.units_c, hdr, w + L.body_c, st, &n, false);
+    if (rc) return rc;
+    launches += n;
+  }
+  // request group: every request is its own single "candidate" with q_r query tokens
+  d.q = a->q_req;
+  d.cand_off_dev = ident;
+  d.cand_off_host = nullptr;
+  d.q_ptr = a->q_r;
+  d.k_ptr = kv + 2 * hd * 2;
+  d.v_ptr = kv + 3 * hd * 2;
+  d.o_ptr = a->o_r;
+  d.lse_ptr = a->lse_r;
+  rc = dca_run(&d, a->R, L.T, L.units_r, hdr, w + L.body_r, st, &n, false);
+  if (rc) return rc;
+  g_last_launches = launches + n;
+  return ROCS_OK;
 }
 
 size_t rocs_proj_workspace_size(const rocs_proj_args* a) {

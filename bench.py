@@ -5,8 +5,9 @@ A step is one pass of the hot path over one batch of synthetic inputs.  Default 
 ("ikbo_step"): IKBO-LCB on the bf16 LCB workload (R=64 requests, N_r ~ U{256..1024},
 n_r=256, n_c=64, d=128, o_r=o_c=128) followed by IKBO-DCA on the long-history workload
 (R=8, L_r ~ U{4096..8192}, H=4, dh=128, 2048 candidates x q=4 per request).  Other
-workloads: "lcb", "dca", "dca_short" (R=32, L=2048, H=8, 512 candidates, q=1) and "chain"
-(LCB -> query projection -> DCA, lognormal candidates per request).
+workloads: "lcb", "dca", "dca_short" (R=32, L=2048, H=8, 512 candidates, q=1), "dca_block"
+(K/V projections once per request + candidate and request attention, Eq. (13) both groups) and
+"chain" (LCB -> query projection -> DCA, lognormal candidates per request).
 
 Reported: TFLOP/s on the non-materialised IKBO formulation (value), per-kernel rooflines
 against MEASURED_PEAKS.json, an end-to-end figure with host<->device copies, the fp64 CPU
@@ -188,6 +189,75 @@ class DcaPart(Part):
         return time.perf_counter() - t0, frac
 
 
+class DcaBlockPart(Part):
+    """Both query groups of Eq. (13): K/V projections once per request + candidate and request attention."""
+    bound, kernel = "tensor", "dca"
+
+    def __init__(self, b: ri.DcaBlockInputs, name="dca_block"):
+        self.b, self.name, self.x = b, name, b
+        self.units = b.C
+
+    def flops(self):
+        b = self.b
+        T, d_s, hd = int(b.seq_off[-1]), b.s_seq.shape[1], b.H * b.dh
+        ident = np.arange(b.R + 1)
+        return (acc.proj_flops(T, 4 * hd, d_s) + acc.dca_flops(b.cand_off, b.seq_off, b.q, b.H, b.dh)
+                + acc.dca_flops(ident, b.seq_off, b.q_req, b.H, b.dh))
+
+    def bytes(self):
+        b = self.b
+        return 2 * (b.s_seq.size + b.w_kv.size + 2 * b.q_c.size + 2 * b.q_r.size) + 4 * (b.C * b.q + b.R * b.q_req) * b.H
+
+    def to_device(self, ikbo, torch, dev):
+        b = self.b
+        self.h_in = [_pin(torch, a) for a in (b.s_seq, b.q_c, b.q_r)]
+        self.d_in = [h.to(dev) for h in self.h_in]
+        self.w = _to_dev(torch, b.w_kv, dev)
+        self.coff = ikbo.offsets(b.cand_off, dev)
+        self.soff = ikbo.offsets(b.seq_off, dev)
+        self.h_offs = [_pin(torch, b.cand_off), _pin(torch, b.seq_off)]
+        s, qc, qr = self.d_in
+        self.outs = list(ikbo.rocs_dca_block_forward(s, self.w, qc, qr, self.coff, self.soff, b.q, b.q_req, b.scale))
+        self.ws = ikbo.rocs_dca_block_forward.last_workspace
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in self.outs]
+
+    def run(self, ikbo):
+        b = self.b
+        s, qc, qr = self.d_in
+        ikbo.rocs_dca_block_forward(s, self.w, qc, qr, self.coff, self.soff, b.q, b.q_req, b.scale,
+                                    o_c=self.outs[0], o_r=self.outs[2], workspace=self.ws)
+        return ikbo.last_launch_count()
+
+    def h2d(self):
+        n = 0
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+            n += h.numel() * h.element_size()
+        for h, d in zip(self.h_offs, (self.coff[0], self.soff[0])):
+            d.copy_(h, non_blocking=True)
+            n += h.numel() * 4
+        return n
+
+    def d2h(self):
+        for h, d in zip(self.h_out, self.outs):
+            h.copy_(d, non_blocking=True)
+        return sum(h.numel() * h.element_size() for h in self.h_out)
+
+    def status(self, ikbo):
+        return ikbo.rocs_read_status(self.ws)
+
+    def oracle_sample(self, oracle, n, seed):
+        b = self.b
+        sel = np.random.RandomState(seed).choice(b.C, size=min(n, b.C), replace=False)
+        L = np.diff(b.seq_off.astype(np.int64))
+        m = np.repeat(np.arange(b.R), np.diff(b.cand_off))
+        frac = float(L[m[sel]].sum()) / float(L[m].sum())
+        t0 = time.perf_counter()
+        oracle.dca_block(b.cand_off, b.seq_off, b.s_seq, *b.weights(), b.q_c, b.q_r, b.q, b.q_req, b.scale,
+                         sel_cand=sel, sel_req=[])
+        return time.perf_counter() - t0, frac
+
+
 class ProjPart(Part):
     bound, kernel = "tensor", "proj"
 
@@ -284,6 +354,8 @@ def make_parts(workload):
         return [DcaPart(ri.dca_long())]
     if workload == "dca_short":
         return [DcaPart(ri.dca_bf16())]
+    if workload == "dca_block":
+        return [DcaBlockPart(ri.dca_block())]
     if workload == "chain":
         ci = ri.chain()
         lcb = LcbPart(ci.lcb, "chain_lcb")
@@ -305,6 +377,9 @@ def workload_config(workload, parts):
         if isinstance(p, LcbPart):
             cfg["parts"][p.name] = {"R": x.R, "C": x.C, "n_r": x.n_r, "n_c": x.n_c, "d": x.d, "o_r": x.o_r,
                                     "o_c": x.o_c, "recipe": x.recipe}
+        elif isinstance(p, DcaBlockPart):
+            cfg["parts"][p.name] = {"R": x.R, "C": x.C, "q": x.q, "q_req": x.q_req, "H": x.H, "dh": x.dh,
+                                    "d_s": int(x.s_seq.shape[1]), "sum_L": int(x.seq_off[-1]), "recipe": x.recipe}
         else:
             cfg["parts"][p.name] = {"R": x.R, "C": x.C, "q": x.q, "H": x.H, "dh": x.dh, "sum_L": x.total_L,
                                     "recipe": x.recipe}
@@ -594,7 +669,8 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ikbo", choices=["ikbo", "reference"])
-    ap.add_argument("--workload", default="ikbo_step", choices=["ikbo_step", "lcb", "dca", "dca_short", "chain"])
+    ap.add_argument("--workload", default="ikbo_step",
+                    choices=["ikbo_step", "lcb", "dca", "dca_short", "dca_block", "chain"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--no-e2e", action="store_true")

@@ -166,6 +166,8 @@ ROCS_API int rocs_lcb_forward_noalloc(const rocs_lcb_args* args, rocs_stream_t s
  * but no keys gets O = 0 and LSE = -inf.  Every query token attends to all keys of its
  * request (non-causal); query tokens of one candidate do not attend to each other.
  * Supported: dh in {64, 128}, H >= 1, q >= 1, row strides multiples of 16 bytes.
+ * kv_ld: row stride of K and V in elements (0 means H*dh, i.e. dense rows); it lets K and V be
+ * read in place from a wider projection output.
  * ---------------------------------------------------------------------------------- */
 typedef struct {
   int64_t R, q, H, dh;
@@ -181,6 +183,7 @@ typedef struct {
   float* lse_ptr;
   void* workspace; /* >= rocs_dca_workspace_size(args): status, work-unit table, counter */
   size_t workspace_bytes;
+  int64_t kv_ld; /* row stride of K and V in elements; 0 = H*dh */
 } rocs_dca_args;
 
 ROCS_API size_t rocs_dca_workspace_size(const rocs_dca_args* args);
@@ -195,6 +198,41 @@ ROCS_API int rocs_dca_forward(const rocs_dca_args* args, rocs_stream_t stream);
  * Workspace: rocs_dca_expand_workspace_size(args, chunk). */
 ROCS_API size_t rocs_dca_expand_workspace_size(const rocs_dca_args* args, int64_t chunk);
 ROCS_API int rocs_dca_forward_expand(const rocs_dca_args* args, int64_t chunk, rocs_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * DCA block: both query groups of section 3.2, Eq. (13), with the K/V projections done once per
+ * request (section 4.1: (S_{m_i}) W = (S W)_{m_i}):
+ *   [K^C | V^C | K^R | V^R] = S . [W_K^C ; W_V^C ; W_K^R ; W_V^R]^T     (one GEMM at batch B_r)
+ *   A^C_i = softmax(scale Q^C_i K^C_{m_i}^T) V^C_{m_i}                   (IKBO-DCA, candidate group)
+ *   A^R_r = softmax(scale Q^R_r K^R_r^T) V^R_r                            (request group, q_req tokens)
+ *   s_seq [T, d_s] bf16     request sequence representation, T = seq_off_host[R]
+ *   w_kv  [4*H*dh, d_s]     the four projection weights stacked in that order
+ *   q_c [C*q, H, dh], q_r [R*q_req, H, dh]; o_c / o_r alike; lse_c [C*q, H], lse_r [R*q_req, H]
+ *   (lse pointers may be NULL).  Projected K/V are stored bf16 in the workspace.
+ * Supported: dh in {64, 128}, d_s % 64 == 0, q >= 1, q_req >= 1.
+ * Launches: one projection GEMM, one identity-map fill and two (schedule + attention) pairs.
+ * ---------------------------------------------------------------------------------- */
+typedef struct {
+  int64_t R, q, q_req, H, dh, d_s; /* q: tokens per candidate, q_req: request query tokens */
+  float scale;
+  const int32_t* cand_off_dev;  /* [R+1] */
+  const int32_t* cand_off_host; /* [R+1] */
+  const int32_t* seq_off_dev;   /* [R+1] */
+  const int32_t* seq_off_host;  /* [R+1] */
+  const void* s_seq;
+  const void* w_kv;
+  const void* q_c;
+  const void* q_r;
+  void* o_c;
+  float* lse_c;
+  void* o_r;
+  float* lse_r;
+  void* workspace; /* >= rocs_dca_block_workspace_size(args) */
+  size_t workspace_bytes;
+} rocs_dca_block_args;
+
+ROCS_API size_t rocs_dca_block_workspace_size(const rocs_dca_block_args* args);
+ROCS_API int rocs_dca_block_forward(const rocs_dca_block_args* args, rocs_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * Linear query projection of the chained block (section 3.2, Eq. (12), plain linear

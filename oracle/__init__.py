@@ -13,6 +13,9 @@ paper-archivist reading notes:
 * :func:`dca` -- section 3.2, Eq. (13), candidate-group cross attention
   ``softmax(scale * Q K^T) V`` over the candidate's own request keys, non-causal,
   K/V copied per candidate.
+* :func:`dca_block` -- section 3.2, Eq. (13) with both query groups: K/V projections of the
+  request sequence (per candidate, broadcast materialised, then rounded to bf16) and the
+  request-group attention A^R next to the candidate-group attention A^C.
 * :func:`proj` / :func:`chain` -- the chained block: LCB output -> bf16 -> linear
   query projection (section 3.2, Eq. (12), read as a plain linear map) -> bf16 -> DCA.
 
@@ -66,6 +69,8 @@ def _L():
         lib.rocs_oracle_proj.argtypes = [i64, i64, i64, vp, vp, vp, i32]
         lib.rocs_oracle_chain.argtypes = [i64, vp, i64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp,
                                           i64, i64, dbl, vp, vp, i64, vp, vp, vp, vp, vp, i32]
+        lib.rocs_oracle_dca_block.argtypes = [i64, vp, vp, i64, i64, i64, i64, i64, dbl, vp, vp, vp, vp, vp, vp, vp,
+                                              i64, vp, vp, vp, i64, vp, vp, vp, i32]
         lib.rocs_oracle_round_bf16.restype = dbl
         lib.rocs_oracle_round_bf16.argtypes = [dbl]
         lib.rocs_oracle_max_threads.restype = i32
@@ -171,3 +176,24 @@ def chain(ci, sel_cand, nthreads: int = 0):
     if rc != ORC_OK:
         raise OracleError(rc)
     return y, qo, o, lse
+
+
+def dca_block(cand_off, seq_off, s_seq, w_kc, w_vc, w_kr, w_vr, q_c, q_r, q: int, q_req: int, scale: float,
+              sel_cand=None, sel_req=None, nthreads: int = 0):
+    """Section 3.2 Eq. (13), both groups.  Returns ``(o_c, lse_c, o_r, lse_r)`` in float64:
+    o_c [n_c, q, H, dh], lse_c [n_c, q, H], o_r [n_r, q_req, H, dh], lse_r [n_r, q_req, H]."""
+    cand_off, seq_off = _c(cand_off, np.int32), _c(seq_off, np.int32)
+    R, C = len(cand_off) - 1, int(cand_off[-1])
+    d_s = s_seq.shape[1]
+    H, dh = q_c.shape[1], q_c.shape[2]
+    sc = np.arange(C, dtype=np.int64) if sel_cand is None else _c(sel_cand, np.int64)
+    sr = np.arange(R, dtype=np.int64) if sel_req is None else _c(sel_req, np.int64)
+    o_c = np.empty((len(sc), q, H, dh)); lse_c = np.empty((len(sc), q, H))
+    o_r = np.empty((len(sr), q_req, H, dh)); lse_r = np.empty((len(sr), q_req, H))
+    arrs = [_c(a, np.uint16) for a in (s_seq, w_kc, w_vc, w_kr, w_vr, q_c, q_r)]
+    rc = _L().rocs_oracle_dca_block(R, _p(cand_off), _p(seq_off), q, q_req, H, dh, d_s, float(scale),
+                                    *[_p(a) for a in arrs], len(sc), _p(sc), _p(o_c), _p(lse_c), len(sr), _p(sr),
+                                    _p(o_r), _p(lse_r), nthreads)
+    if rc != ORC_OK:
+        raise OracleError(rc)
+    return o_c, lse_c, o_r, lse_r

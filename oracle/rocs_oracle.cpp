@@ -318,6 +318,63 @@ int rocs_oracle_chain(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n
   return bad ? ORC_ISOLATION : ORC_OK;
 }
 
+// DCA block (section 3.2, Eq. (13)), both query groups, for the selected requests / candidates.
+// s_seq [T, d_s] bf16 request sequence representation (rows seq_off[r]..seq_off[r+1]-1 belong to r);
+// w_kc, w_vc, w_kr, w_vr [H*dh, d_s] bf16; q_c [C*q, H, dh] and q_r [R*q_r, H, dh] bf16.
+// Candidate group: for candidate i the request's sequence rows are copied (materialised broadcast),
+// projected K_i = S_{m_i} W_K^C^T, V_i = S_{m_i} W_V^C^T in fp64, rounded to bf16 (the stored
+// precision of projected K/V), and attended by the candidate's q tokens.  Request group: the same
+// with W_K^R, W_V^R and request r's own q_r tokens.  Outputs o_c [n_sel_c, q, H, dh], lse_c
+// [n_sel_c, q, H], o_r [n_sel_r, q_r, H, dh], lse_r [n_sel_r, q_r, H].
+static void project_rows(const uint16_t* s_seq, int64_t s0, int64_t L, int64_t d_s, const uint16_t* w, int64_t n_out,
+                         std::vector<uint16_t>& out) {
+  out.assign((size_t)(L * n_out), 0);
+  for (int64_t j = 0; j < L; ++j)
+    for (int64_t n = 0; n < n_out; ++n) {
+      double acc = 0.0;
+      for (int64_t e = 0; e < d_s; ++e) acc += widen(s_seq, 1, (s0 + j) * d_s + e) * widen(w, 1, n * d_s + e);
+      const float f = (float)round_bf16(acc);  // exact: a bf16 value
+      uint32_t u;
+      std::memcpy(&u, &f, 4);
+      out[(size_t)(j * n_out + n)] = (uint16_t)(u >> 16);
+    }
+}
+
+int rocs_oracle_dca_block(int64_t R, const int32_t* cand_off, const int32_t* seq_off, int64_t q, int64_t q_r,
+                          int64_t H, int64_t dh, int64_t d_s, double scale, const uint16_t* s_seq, const uint16_t* w_kc,
+                          const uint16_t* w_vc, const uint16_t* w_kr, const uint16_t* w_vr, const uint16_t* q_c,
+                          const uint16_t* q_rq, int64_t n_sel_c, const int64_t* sel_c, double* o_c, double* lse_c,
+                          int64_t n_sel_r, const int64_t* sel_r, double* o_r, double* lse_r, int nthreads) {
+  if (q < 0 || q_r < 0 || H < 0 || dh < 0 || d_s < 0) return ORC_INVALID;
+  if (!csr_ok(cand_off, R, -1) || !csr_ok(seq_off, R, -1)) return ORC_BAD_OFFSETS;
+  set_threads(nthreads);
+  const int64_t C = cand_off[R], n_out = H * dh;
+  for (int64_t k = 0; k < n_sel_c; ++k)
+    if (sel_c[k] < 0 || sel_c[k] >= C) return ORC_INVALID;
+  for (int64_t k = 0; k < n_sel_r; ++k)
+    if (sel_r[k] < 0 || sel_r[k] >= R) return ORC_INVALID;
+  std::vector<int64_t> m = index_map(cand_off, R);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t k = 0; k < n_sel_c; ++k) {
+    const int64_t i = sel_c[k], r = m[(size_t)i], s0 = seq_off[r], L = seq_off[r + 1] - s0;
+    std::vector<uint16_t> Kp, Vp;  // this candidate's own copy of the projected request sequence
+    project_rows(s_seq, s0, L, d_s, w_kc, n_out, Kp);
+    project_rows(s_seq, s0, L, d_s, w_vc, n_out, Vp);
+    const DcaDims D{q, H, dh, scale};
+    dca_candidate(D, q_c, Kp.data(), Vp.data(), i, 0, L, nullptr, o_c + k * q * n_out, lse_c + k * q * H);
+  }
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t k = 0; k < n_sel_r; ++k) {
+    const int64_t r = sel_r[k], s0 = seq_off[r], L = seq_off[r + 1] - s0;
+    std::vector<uint16_t> Kp, Vp;
+    project_rows(s_seq, s0, L, d_s, w_kr, n_out, Kp);
+    project_rows(s_seq, s0, L, d_s, w_vr, n_out, Vp);
+    const DcaDims D{q_r, H, dh, scale};
+    dca_candidate(D, q_rq, Kp.data(), Vp.data(), r, 0, L, nullptr, o_r + k * q_r * n_out, lse_r + k * q_r * H);
+  }
+  return ORC_OK;
+}
+
 // Exposed for the oracle's own tests of its bf16 rounding.
 double rocs_oracle_round_bf16(double x) { return round_bf16(x); }
 

@@ -33,6 +33,7 @@ _LIB = os.path.join(_HERE, "librocs_gen.so")
 
 # one stream id per tensor role
 S_XREQ, S_XCAND, S_WRR, S_WCR, S_WCC, S_NCAND, S_LSEQ, S_Q, S_K, S_V, S_WQ = range(1, 12)
+S_SEQ, S_WKV, S_QREQ = range(12, 15)
 
 
 def build_lib(force: bool = False) -> str:
@@ -247,3 +248,52 @@ def chain(seed: int = 5, R: int = 128, median: float = 512.0, sigma: float = 1.0
     ci.recipe = (f"R={R}, N_r~round(lognormal(ln {median:g}, {sigma:g})) clipped {clip}; LCB n_r=512, n_c=128, d=128, "
                  f"o_r=o_c=128; W_q [{H*dh}x{n_in}] ~N(0,1/{n_in}); DCA H={H}, dh={dh}, q=1, L_r~U{{{Llo}..{Lhi}}}")
     return ci
+
+
+@dataclass
+class DcaBlockInputs:
+    """Inputs of the DCA block (section 3.2, Eq. (13), both query groups)."""
+    name: str
+    cand_off: np.ndarray
+    seq_off: np.ndarray
+    q: int
+    q_req: int
+    H: int
+    dh: int
+    scale: float
+    s_seq: np.ndarray  # uint16 [T, d_s] request sequence representation
+    w_kv: np.ndarray  # uint16 [4*H*dh, d_s]: W_K^C, W_V^C, W_K^R, W_V^R stacked
+    q_c: np.ndarray  # uint16 [C*q, H, dh]
+    q_r: np.ndarray  # uint16 [R*q_req, H, dh]
+    recipe: str = ""
+
+    @property
+    def R(self):
+        return len(self.cand_off) - 1
+
+    @property
+    def C(self):
+        return int(self.cand_off[-1])
+
+    def weights(self):
+        n = self.H * self.dh
+        return [self.w_kv[k * n:(k + 1) * n] for k in range(4)]
+
+
+def make_dca_block(name, counts, lengths, q, q_req, H, dh, d_s, seed) -> DcaBlockInputs:
+    """S ~ N(0,1); projection weights ~ N(0, 1/d_s); queries ~ N(0,1)."""
+    coff, soff = counts_to_offsets(counts), counts_to_offsets(lengths)
+    R, C, T = len(counts), int(coff[-1]), int(soff[-1])
+    return DcaBlockInputs(name=name, cand_off=coff, seq_off=soff, q=q, q_req=q_req, H=H, dh=dh,
+                          scale=1.0 / math.sqrt(dh), s_seq=normal(seed, S_SEQ, (T, d_s)),
+                          w_kv=normal(seed, S_WKV, (4 * H * dh, d_s), 1.0 / math.sqrt(d_s)),
+                          q_c=normal(seed, S_Q, (C * q, H, dh)), q_r=normal(seed, S_QREQ, (R * q_req, H, dh)))
+
+
+def dca_block(seed: int = 6, R: int = 8, lo: int = 4096, hi: int = 8192, H: int = 4, dh: int = 128, d_s: int = 256,
+              n_cand: int = 2048, q: int = 4, q_req: int = 64) -> DcaBlockInputs:
+    lengths = uniform_int(seed, S_LSEQ, lo, hi, R)
+    x = make_dca_block("dca_block", [n_cand] * R, lengths, q, q_req, H, dh, d_s, seed)
+    x.recipe = (f"R={R}, L_r~U{{{lo}..{hi}}}, d_s={d_s}, H={H}, dh={dh}, N_r={n_cand}, q={q}, request queries "
+                f"q_req={q_req}; S,Q~N(0,1), W~N(0,1/d_s)")
+    return x

@@ -374,3 +374,53 @@ def test_dca_large_scores_stable(oracle_mod):
     w0 = 1.0 / (1.0 + math.exp(-4.0))
     assert abs(o.item() - w0) <= 1e-12
     assert abs(lse.item() - (800.0 + math.log1p(math.exp(-4.0)))) <= 1e-12
+
+
+# ------------------------------------------------------------------------------ DCA block (both groups)
+def _block_inputs(seed, counts, lengths, q=2, q_req=3, H=2, dh=8, d_s=16):
+    coff, soff = ri.counts_to_offsets(counts), ri.counts_to_offsets(lengths)
+    R, C, T = len(counts), int(coff[-1]), int(soff[-1])
+    g = lambda stream, shape, std=1.0: ri.normal(seed, stream, shape, std)
+    return dict(cand_off=coff, seq_off=soff, s_seq=g(40, (T, d_s)), w_kc=g(41, (H * dh, d_s), 0.25),
+                w_vc=g(42, (H * dh, d_s), 0.25), w_kr=g(43, (H * dh, d_s), 0.25), w_vr=g(44, (H * dh, d_s), 0.25),
+                q_c=g(45, (C * q, H, dh)), q_r=g(46, (R * q_req, H, dh)), q=q, q_req=q_req, scale=1.0 / math.sqrt(dh))
+
+
+def _project_bf16(oracle_mod, s_seq, w):
+    """K = S W^T with a library matmul in float64, then the oracle's (separately pinned) bf16 rounding."""
+    k = ri.bf16_to_f32(s_seq).astype(np.float64) @ ri.bf16_to_f32(w).astype(np.float64).T
+    kb = np.vectorize(oracle_mod.round_bf16)(k).astype(np.float32)
+    return (kb.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_dca_block_equals_projection_then_attention(oracle_mod):
+    """Eq. (13): A^C = Attn(Q^C, S W_K^C, S W_V^C) and A^R = Attn(Q^R, S W_K^R, S W_V^R).  The block
+    oracle projects a per-candidate copy of S (broadcast first); here S is projected once per request
+    with a library matmul (projection first, section 4.1) and fed to the pinned attention oracle."""
+    b = _block_inputs(51, [2, 0, 3], [5, 7, 4])
+    H, dh = b["q_c"].shape[1], b["q_c"].shape[2]
+    o_c, l_c, o_r, l_r = oracle_mod.dca_block(b["cand_off"], b["seq_off"], b["s_seq"], b["w_kc"], b["w_vc"],
+                                              b["w_kr"], b["w_vr"], b["q_c"], b["q_r"], b["q"], b["q_req"], b["scale"])
+    kc, vc = (_project_bf16(oracle_mod, b["s_seq"], w).reshape(-1, H, dh) for w in (b["w_kc"], b["w_vc"]))
+    oo, ll = oracle_mod.dca(b["cand_off"], b["seq_off"], b["q_c"], kc, vc, b["q"], b["scale"])
+    assert np.array_equal(o_c, oo) and np.array_equal(l_c, ll)
+    kr, vr = (_project_bf16(oracle_mod, b["s_seq"], w).reshape(-1, H, dh) for w in (b["w_kr"], b["w_vr"]))
+    R = len(b["cand_off"]) - 1
+    ident = np.arange(R + 1, dtype=np.int32)  # every request attends over its own keys with its own queries
+    oo, ll = oracle_mod.dca(ident, b["seq_off"], b["q_r"], kr, vr, b["q_req"], b["scale"])
+    assert np.array_equal(o_r, oo) and np.array_equal(l_r, ll)
+
+
+def test_dca_block_closed_forms(oracle_mod):
+    """W_K = 0: uniform weights, O = mean over the request's keys of the projected V.
+    A single key: O = that key's projected V exactly."""
+    b = _block_inputs(52, [3, 2], [6, 1])
+    H, dh = b["q_c"].shape[1], b["q_c"].shape[2]
+    zero = np.zeros_like(b["w_kc"])
+    o_c, _, o_r, _ = oracle_mod.dca_block(b["cand_off"], b["seq_off"], b["s_seq"], zero, b["w_vc"], zero,
+                                          b["w_vr"], b["q_c"], b["q_r"], b["q"], b["q_req"], b["scale"])
+    vc = ri.bf16_to_f32(_project_bf16(oracle_mod, b["s_seq"], b["w_vc"])).astype(np.float64).reshape(-1, H, dh)
+    vr = ri.bf16_to_f32(_project_bf16(oracle_mod, b["s_seq"], b["w_vr"])).astype(np.float64).reshape(-1, H, dh)
+    assert np.abs(o_c[:3] - vc[0:6].mean(0)).max() <= 1e-12
+    assert np.abs(o_c[3:] - vc[6]).max() <= 1e-12
+    assert np.abs(o_r[0] - vr[0:6].mean(0)).max() <= 1e-12 and np.abs(o_r[1] - vr[6]).max() <= 1e-12
