@@ -16,6 +16,9 @@ paper-archivist reading notes:
 * :func:`dca_block` -- section 3.2, Eq. (13) with both query groups: K/V projections of the
   request sequence (per candidate, broadcast materialised, then rounded to bf16) and the
   request-group attention A^R next to the candidate-group attention A^C.
+* :func:`lcb_block` -- section 3.1.2 Eq. (4)-(6) with section 3.1.3 Eq. (7)-(8): the LCB with a
+  per-row bias, a residual merge, a group-local LayerNorm/RMSNorm over d and an activation, each
+  output group with its own parameters (broadcast materialised as in :func:`lcb`).
 * :func:`proj` / :func:`chain` -- the chained block: LCB output -> bf16 -> linear
   query projection (section 3.2, Eq. (12), read as a plain linear map) -> bf16 -> DCA.
 
@@ -36,6 +39,17 @@ _SRC = os.path.join(_HERE, "rocs_oracle.cpp")
 _LIB = os.path.join(_HERE, "librocs_oracle.so")
 
 ORC_OK, ORC_INVALID, ORC_BAD_OFFSETS, ORC_ISOLATION = 0, 1, 2, 10
+
+
+class Epi(ctypes.Structure):
+    """One output group's epilogue; the fields mirror ``OrcEpi`` in rocs_oracle.cpp."""
+    _fields_ = [("bias", ctypes.c_void_p), ("residual", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("eps", ctypes.c_double), ("norm", ctypes.c_int32),
+                ("act", ctypes.c_int32)]
+
+
+NORMS = {"none": 0, "layernorm": 1, "rmsnorm": 2}
+ACTS = {"none": 0, "relu": 1, "silu": 2, "gelu": 3}
 
 
 class OracleError(RuntimeError):
@@ -71,6 +85,8 @@ def _L():
                                           i64, i64, dbl, vp, vp, i64, vp, vp, vp, vp, vp, i32]
         lib.rocs_oracle_dca_block.argtypes = [i64, vp, vp, i64, i64, i64, i64, i64, dbl, vp, vp, vp, vp, vp, vp, vp,
                                               i64, vp, vp, vp, i64, vp, vp, vp, i32]
+        lib.rocs_oracle_lcb_block.argtypes = [i64, vp, i64, i64, i64, i64, i64, vp, vp, vp, vp, vp,
+                                              ctypes.POINTER(Epi), ctypes.POINTER(Epi), i64, vp, vp, i64, vp, vp, i32]
         lib.rocs_oracle_round_bf16.restype = dbl
         lib.rocs_oracle_round_bf16.argtypes = [dbl]
         lib.rocs_oracle_max_threads.restype = i32
@@ -197,3 +213,40 @@ def dca_block(cand_off, seq_off, s_seq, w_kc, w_vc, w_kr, w_vr, q_c, q_r, q: int
     if rc != ORC_OK:
         raise OracleError(rc)
     return o_c, lse_c, o_r, lse_r
+
+
+def _epi(e, keep):
+    """``e``: object with bias/residual/gamma/beta (arrays or None), eps, norm, act (names or codes)."""
+    def arr(a, dt):
+        if a is None:
+            return None
+        a = _c(a, dt)
+        keep.append(a)
+        return a.ctypes.data
+    norm = NORMS[e.norm] if isinstance(e.norm, str) else int(e.norm)
+    act = ACTS[e.act] if isinstance(e.act, str) else int(e.act)
+    return Epi(arr(e.bias, np.float32), arr(e.residual, np.uint16), arr(e.gamma, np.float32),
+               arr(e.beta, np.float32), float(e.eps), norm, act)
+
+
+def lcb_block(cand_off, x_req, x_cand, w_rr, w_cr, w_cc, epi_r, epi_c, sel_req=None, sel_cand=None,
+              nthreads: int = 0):
+    """LCB block with per-group epilogues (bf16 inputs).  Returns ``(y_req, y_cand)`` in float64."""
+    cand_off = _c(cand_off, np.int32)
+    R, C = len(cand_off) - 1, int(cand_off[-1])
+    _, n_r, d = x_req.shape
+    n_c = x_cand.shape[1]
+    o_r, o_c = w_rr.shape[0], w_cc.shape[0]
+    sel_req = np.arange(R, dtype=np.int64) if sel_req is None else _c(sel_req, np.int64)
+    sel_cand = np.arange(C, dtype=np.int64) if sel_cand is None else _c(sel_cand, np.int64)
+    y_req = np.empty((len(sel_req), o_r, d), dtype=np.float64)
+    y_cand = np.empty((len(sel_cand), o_c, d), dtype=np.float64)
+    keep = []
+    er, ec = _epi(epi_r, keep), _epi(epi_c, keep)
+    arrs = [_c(a, np.uint16) for a in (x_req, x_cand, w_rr, w_cr, w_cc)]
+    rc = _L().rocs_oracle_lcb_block(R, _p(cand_off), n_r, n_c, d, o_r, o_c, *[_p(a) for a in arrs],
+                                    ctypes.byref(er), ctypes.byref(ec), len(sel_req), _p(sel_req), _p(y_req),
+                                    len(sel_cand), _p(sel_cand), _p(y_cand), nthreads)
+    if rc != ORC_OK:
+        raise OracleError(rc)
+    return y_req, y_cand

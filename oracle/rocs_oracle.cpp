@@ -201,6 +201,73 @@ void dca_candidate(const DcaDims& D, const uint16_t* Q, const uint16_t* K, const
     }
 }
 
+// ---- LCB block: bias, group-local norm and pointwise epilogue --------------------------
+// One output group's epilogue (the fields mirror the ctypes structure in oracle/__init__.py).
+//   bias     [o] fp32, per output row, broadcast over d: the GLM linear bias of section 3.1.2,
+//            Eq. (4), applied on the row axis of the LCB (null = none)
+//   residual bf16 rows of the group's output shape (null = none): a pointwise merge of an
+//            aligned input of the same group, section 3.1.3, Eq. (8)
+//   norm     0 none, 1 LayerNorm, 2 RMSNorm over the d entries of one output row, with the
+//            group's own gamma/beta [d] (null = 1 / 0): the group-local norm of Eq. (7)
+//   act      0 none, 1 ReLU, 2 SiLU, 3 GELU (erf form): a pointwise activation, Eq. (8)
+// Order on one output row y: y = W x + b; y += residual; y = Norm(y); y = act(y).
+struct OrcEpi {
+  const float* bias;
+  const uint16_t* residual;
+  const float* gamma;
+  const float* beta;
+  double eps;
+  int32_t norm;
+  int32_t act;
+};
+
+double activation(int act, double x) {
+  switch (act) {
+    case 1: return x > 0.0 ? x : 0.0;
+    case 2: return x / (1.0 + std::exp(-x));
+    case 3: return 0.5 * x * (1.0 + std::erf(x / std::sqrt(2.0)));
+    default: return x;
+  }
+}
+
+// y [d]: one output row of a group; res_row = index of this row in the group's residual
+void epilogue_row(const OrcEpi& e, int64_t d, int64_t res_row, double* y) {
+  if (e.residual)
+    for (int64_t c = 0; c < d; ++c) y[c] += widen(e.residual, 1, res_row * d + c);
+  if (e.norm == 1 || e.norm == 2) {
+    double mean = 0.0;
+    if (e.norm == 1) {
+      for (int64_t c = 0; c < d; ++c) mean += y[c];
+      mean /= (double)d;
+    }
+    double var = 0.0;  // LayerNorm: population variance; RMSNorm: mean square
+    for (int64_t c = 0; c < d; ++c) var += (y[c] - mean) * (y[c] - mean);
+    var /= (double)d;
+    const double inv = 1.0 / std::sqrt(var + e.eps);
+    for (int64_t c = 0; c < d; ++c) {
+      const double g = e.gamma ? (double)e.gamma[c] : 1.0, b = e.beta ? (double)e.beta[c] : 0.0;
+      y[c] = (y[c] - mean) * inv * g + b;
+    }
+  }
+  for (int64_t c = 0; c < d; ++c) y[c] = activation(e.act, y[c]);
+}
+
+bool epi_ok(const OrcEpi* e) {
+  return e && e->norm >= 0 && e->norm <= 2 && e->act >= 0 && e->act <= 3 && e->eps >= 0.0;
+}
+
+// Y^R_r of the block: W_RR X^R_r + b^R, then the request epilogue
+void lcb_block_request(const LcbDims& D, const void* x_req, const std::vector<double>& W, const OrcEpi& er,
+                       int64_t r, double* y) {
+  lcb_request(D, 1, x_req, W, r, y);
+  for (int64_t o = 0; o < D.o_r; ++o) {
+    double* row = y + o * D.d;
+    if (er.bias)
+      for (int64_t c = 0; c < D.d; ++c) row[c] += (double)er.bias[o];
+    epilogue_row(er, D.d, r * D.o_r + o, row);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -373,6 +440,60 @@ int rocs_oracle_dca_block(int64_t R, const int32_t* cand_off, const int32_t* seq
     dca_candidate(D, q_rq, Kp.data(), Vp.data(), r, 0, L, nullptr, o_r + k * q_r * n_out, lse_r + k * q_r * H);
   }
   return ORC_OK;
+}
+
+// LCB block (section 3.1.2 Eq. (4)-(6) with the epilogues of section 3.1.3 Eq. (7)-(8)), bf16 inputs.
+// Each selected candidate's full output [Y^R; Y^C] = W_full X_full + [b^R; b^C] is formed with the
+// broadcast materialised (as rocs_oracle_lcb), then each output row gets its own group's epilogue
+// (residual^R indexed by request row r*o_r+o, residual^C by candidate row i*o_c+o).  The request rows
+// of every candidate's full output must equal Y^R of the request computed alone (Eq. (11)).
+int rocs_oracle_lcb_block(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n_c, int64_t d, int64_t o_r,
+                          int64_t o_c, const uint16_t* x_req, const uint16_t* x_cand, const uint16_t* w_rr,
+                          const uint16_t* w_cr, const uint16_t* w_cc, const OrcEpi* epi_r, const OrcEpi* epi_c,
+                          int64_t n_sel_req, const int64_t* sel_req, double* y_req, int64_t n_sel_cand,
+                          const int64_t* sel_cand, double* y_cand, int nthreads) {
+  if (n_r < 0 || n_c < 0 || d < 0 || o_r < 0 || o_c < 0 || !epi_ok(epi_r) || !epi_ok(epi_c)) return ORC_INVALID;
+  if (!csr_ok(cand_off, R, -1)) return ORC_BAD_OFFSETS;
+  set_threads(nthreads);
+  const LcbDims D{n_r, n_c, d, o_r, o_c};
+  const int64_t C = cand_off[R];
+  for (int64_t k = 0; k < n_sel_req; ++k)
+    if (sel_req[k] < 0 || sel_req[k] >= R) return ORC_INVALID;
+  for (int64_t k = 0; k < n_sel_cand; ++k)
+    if (sel_cand[k] < 0 || sel_cand[k] >= C) return ORC_INVALID;
+  std::vector<int64_t> m = index_map(cand_off, R);
+  std::vector<double> W;
+  lcb_full_weight(D, 1, w_rr, w_cr, w_cc, W);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t k = 0; k < n_sel_req; ++k) lcb_block_request(D, x_req, W, *epi_r, sel_req[k], y_req + k * o_r * d);
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t k = 0; k < n_sel_cand; ++k) {
+    const int64_t i = sel_cand[k], r = m[(size_t)i], ni = n_r + n_c, no = o_r + o_c;
+    // the explicit broadcast: X_full = [X^R_r ; X^C_i]
+    std::vector<double> X((size_t)(ni * d)), Y((size_t)(no * d));
+    for (int64_t j = 0; j < n_r; ++j)
+      for (int64_t c = 0; c < d; ++c) X[(size_t)(j * d + c)] = widen(x_req, 1, (r * n_r + j) * d + c);
+    for (int64_t j = 0; j < n_c; ++j)
+      for (int64_t c = 0; c < d; ++c) X[(size_t)((n_r + j) * d + c)] = widen(x_cand, 1, (i * n_c + j) * d + c);
+    for (int64_t o = 0; o < no; ++o) {
+      const double b = o < o_r ? (epi_r->bias ? (double)epi_r->bias[o] : 0.0)
+                               : (epi_c->bias ? (double)epi_c->bias[o - o_r] : 0.0);
+      for (int64_t c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < ni; ++j) acc += W[(size_t)(o * ni + j)] * X[(size_t)(j * d + c)];
+        Y[(size_t)(o * d + c)] = acc + b;
+      }
+      if (o < o_r) epilogue_row(*epi_r, d, r * o_r + o, &Y[(size_t)(o * d)]);
+      else epilogue_row(*epi_c, d, i * o_c + (o - o_r), &Y[(size_t)(o * d)]);
+    }
+    std::vector<double> yr((size_t)(o_r * d));
+    lcb_block_request(D, x_req, W, *epi_r, r, yr.data());
+    for (int64_t e = 0; e < o_r * d; ++e)
+      if (Y[(size_t)e] != yr[(size_t)e]) bad |= 1;
+    for (int64_t e = 0; e < o_c * d; ++e) y_cand[k * o_c * d + e] = Y[(size_t)(o_r * d + e)];
+  }
+  return bad ? ORC_ISOLATION : ORC_OK;
 }
 
 // Exposed for the oracle's own tests of its bf16 rounding.

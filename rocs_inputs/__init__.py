@@ -34,6 +34,9 @@ _LIB = os.path.join(_HERE, "librocs_gen.so")
 # one stream id per tensor role
 S_XREQ, S_XCAND, S_WRR, S_WCR, S_WCC, S_NCAND, S_LSEQ, S_Q, S_K, S_V, S_WQ = range(1, 12)
 S_SEQ, S_WKV, S_QREQ = range(12, 15)
+# epilogue parameters, one stream per (group, role): request group 20.., candidate group 30..
+S_EPI_R, S_EPI_C = 20, 30
+E_BIAS, E_GAMMA, E_BETA, E_RES = range(4)
 
 
 def build_lib(force: bool = False) -> str:
@@ -296,4 +299,62 @@ def dca_block(seed: int = 6, R: int = 8, lo: int = 4096, hi: int = 8192, H: int 
     x = make_dca_block("dca_block", [n_cand] * R, lengths, q, q_req, H, dh, d_s, seed)
     x.recipe = (f"R={R}, L_r~U{{{lo}..{hi}}}, d_s={d_s}, H={H}, dh={dh}, N_r={n_cand}, q={q}, request queries "
                 f"q_req={q_req}; S,Q~N(0,1), W~N(0,1/d_s)")
+    return x
+
+
+# ---- LCB block: the LCB with per-group bias / residual / norm / activation --------------
+@dataclass
+class Epilogue:
+    """One output group's epilogue parameters (section 3.1.2 Eq. 4 bias, section 3.1.3 Eq. 7-8).
+
+    ``bias [o]`` fp32 per output row; ``residual`` bf16 bits with the group's output shape;
+    ``gamma / beta [d]`` fp32; ``norm`` in {"none", "layernorm", "rmsnorm"}; ``act`` in
+    {"none", "relu", "silu", "gelu"}.  Any array may be None (no bias / residual, gamma 1, beta 0).
+    """
+    bias: np.ndarray | None = None
+    residual: np.ndarray | None = None
+    gamma: np.ndarray | None = None
+    beta: np.ndarray | None = None
+    eps: float = 1e-5
+    norm: str = "none"
+    act: str = "none"
+
+
+@dataclass
+class LcbBlockInputs:
+    name: str
+    lcb: LcbInputs
+    epi_r: Epilogue
+    epi_c: Epilogue
+    recipe: str = ""
+
+
+def make_epilogue(seed: int, group_stream: int, o: int, d: int, rows: int, norm: str, act: str,
+                  bias: bool = True, residual: bool = True, affine: bool = True, eps: float = 1e-5) -> Epilogue:
+    """bias ~ N(0, 0.5^2); gamma ~ 1 + N(0, 0.1^2); beta ~ N(0, 0.1^2) (fp32); residual ~ N(0,1) bf16 [rows, o, d]."""
+    g = group_stream
+    return Epilogue(
+        bias=normal(seed, g + E_BIAS, (o,), 0.5, "f32") if bias else None,
+        residual=normal(seed, g + E_RES, (rows, o, d)) if residual else None,
+        gamma=(1.0 + normal(seed, g + E_GAMMA, (d,), 0.1, "f32")).astype(np.float32) if affine else None,
+        beta=normal(seed, g + E_BETA, (d,), 0.1, "f32") if affine else None,
+        eps=eps, norm=norm, act=act)
+
+
+def make_lcb_block(name, counts, n_r, n_c, d, o_r, o_c, seed, norm="layernorm", act="silu", residual=True,
+                   norm_r=None, act_r=None) -> LcbBlockInputs:
+    lcb = make_lcb(name, counts, n_r, n_c, d, o_r, o_c, seed, "bf16")
+    R, C = lcb.R, lcb.C
+    return LcbBlockInputs(
+        name=name, lcb=lcb,
+        epi_r=make_epilogue(seed, S_EPI_R, o_r, d, R, norm_r or norm, act_r or act, residual=residual),
+        epi_c=make_epilogue(seed, S_EPI_C, o_c, d, C, norm, act, residual=residual))
+
+
+def lcb_block(seed: int = 7, R: int = 64, lo: int = 256, hi: int = 1024, residual: bool = True) -> LcbBlockInputs:
+    counts = uniform_int(seed, S_NCAND, lo, hi, R)
+    x = make_lcb_block("lcb_block", counts, 256, 64, 128, 128, 128, seed, "layernorm", "silu", residual)
+    x.recipe = (f"LCB as lcb_bf16 (R={R}, N_r~U{{{lo}..{hi}}}; n_r=256, n_c=64, d=128, o_r=o_c=128) with, per "
+                f"group, bias~N(0,0.25), {'residual~N(0,1) bf16, ' if residual else ''}LayerNorm over d "
+                f"(gamma~1+N(0,0.01), beta~N(0,0.01), eps 1e-5), SiLU; seed {seed}")
     return x

@@ -424,3 +424,123 @@ def test_dca_block_closed_forms(oracle_mod):
     assert np.abs(o_c[:3] - vc[0:6].mean(0)).max() <= 1e-12
     assert np.abs(o_c[3:] - vc[6]).max() <= 1e-12
     assert np.abs(o_r[0] - vr[0:6].mean(0)).max() <= 1e-12 and np.abs(o_r[1] - vr[6]).max() <= 1e-12
+
+
+# ------------------------------------------------------------------------------ LCB block (f4)
+# Section 3.1.2 Eq. (4) (bias), section 3.1.3 Eq. (7) (group-local norm) and Eq. (8) (pointwise
+# merge / activation).  Library routines (numpy matmul, torch layer_norm / rms_norm / silu / gelu
+# in fp64) and closed forms pin the oracle's epilogue.
+def _blk(seed, counts=(3, 0, 2, 1), n_r=5, n_c=3, d=16, o_r=4, o_c=6, norm="layernorm", act="silu", **kw):
+    return ri.make_lcb_block("t", list(counts), n_r, n_c, d, o_r, o_c, seed, norm, act, **kw)
+
+
+def _blk_run(oracle_mod, x, **kw):
+    L = x.lcb
+    return oracle_mod.lcb_block(L.cand_off, L.x_req, L.x_cand, L.w_rr, L.w_cr, L.w_cc, x.epi_r, x.epi_c, **kw)
+
+
+def _library_block(x):
+    """numpy matmul (Eq. 14 form) + torch fp64 norm / activation, straight from the definitions."""
+    import torch.nn.functional as F
+    L = x.lcb
+    w = lambda a: ri.bf16_to_f32(a).astype(np.float64)
+    xr, xc = w(L.x_req), w(L.x_cand)
+    m = np.repeat(np.arange(L.R), np.diff(L.cand_off))
+    yr = np.einsum("on,rnd->rod", w(L.w_rr), xr)
+    yc = np.einsum("on,ind->iod", w(L.w_cr), xr[m]) + np.einsum("on,ind->iod", w(L.w_cc), xc)
+    out = []
+    for y, e in ((yr, x.epi_r), (yc, x.epi_c)):
+        if e.bias is not None:
+            y = y + e.bias.astype(np.float64)[None, :, None]
+        if e.residual is not None:
+            y = y + w(e.residual)
+        t = torch.from_numpy(y)
+        g = None if e.gamma is None else torch.from_numpy(e.gamma.astype(np.float64))
+        b = None if e.beta is None else torch.from_numpy(e.beta.astype(np.float64))
+        if e.norm == "layernorm":
+            t = F.layer_norm(t, (t.shape[-1],), g, b, e.eps)
+        elif e.norm == "rmsnorm":
+            t = F.rms_norm(t, (t.shape[-1],), g, e.eps)
+            if b is not None:
+                t = t + b
+        t = {"none": lambda v: v, "relu": F.relu, "silu": F.silu, "gelu": F.gelu}[e.act](t)
+        out.append(t.numpy())
+    return out
+
+
+@pytest.mark.parametrize("norm,act", [("layernorm", "silu"), ("rmsnorm", "gelu"), ("none", "relu"),
+                                      ("layernorm", "none")])
+def test_lcb_block_matches_library(oracle_mod, norm, act):
+    x = _blk(11, norm=norm, act=act)
+    yr, yc = _blk_run(oracle_mod, x)
+    lr, lc = _library_block(x)
+    for a, b in ((yr, lr), (yc, lc)):
+        assert np.max(np.abs(a - b)) <= 1e-12 * max(1.0, np.max(np.abs(b)))
+
+
+def test_lcb_block_groups_use_their_own_parameters(oracle_mod):
+    # request group RMSNorm + GELU, candidate group LayerNorm + ReLU: a swapped group fails the library check
+    x = _blk(12, norm="layernorm", act="relu", norm_r="rmsnorm", act_r="gelu")
+    yr, yc = _blk_run(oracle_mod, x)
+    lr, lc = _library_block(x)
+    assert np.max(np.abs(yr - lr)) <= 1e-12 * np.max(np.abs(lr))
+    assert np.max(np.abs(yc - lc)) <= 1e-12 * np.max(np.abs(lc))
+
+
+def test_lcb_block_bias_and_residual_closed_forms(oracle_mod):
+    x = _blk(13, norm="none", act="none")
+    L = x.lcb
+    for a in (L.w_rr, L.w_cr, L.w_cc):
+        a[...] = 0
+    yr, yc = _blk_run(oracle_mod, x)
+    # W = 0: Y = b (broadcast over d) + residual, exactly
+    assert np.array_equal(yr, x.epi_r.bias.astype(np.float64)[None, :, None] + ri.bf16_to_f32(x.epi_r.residual))
+    assert np.array_equal(yc, x.epi_c.bias.astype(np.float64)[None, :, None] + ri.bf16_to_f32(x.epi_c.residual))
+
+
+def test_lcb_block_activation_closed_forms(oracle_mod):
+    # W = 0, no residual / norm: every output entry of row o is act(b[o]), so b picks the arguments
+    vals = np.array([0.0, 1.0, -1.0, math.log(3.0), -math.log(3.0), 2.5], dtype=np.float32)
+    res = {}
+    for act in ("relu", "silu", "gelu"):
+        x = _blk(14, norm="none", act=act, residual=False, o_c=len(vals))
+        for a in (x.lcb.w_rr, x.lcb.w_cr, x.lcb.w_cc):
+            a[...] = 0
+        x.epi_c.bias = vals.copy()
+        _, yc = _blk_run(oracle_mod, x)
+        res[act] = yc[0, :, 0]
+        assert np.all(yc == yc[:, :, :1])  # broadcast over d and candidates
+    v = vals.astype(np.float64)
+    assert np.array_equal(res["relu"], np.maximum(v, 0.0))
+    # odd-part identities: f(x) - f(-x) = x for SiLU and GELU (sigma(x)+sigma(-x) = Phi(x)+Phi(-x) = 1)
+    for act in ("silu", "gelu"):
+        assert abs(res[act][1] - res[act][2] - 1.0) <= 1e-15
+        assert abs(res[act][3] - res[act][4] - v[3]) <= 1e-15
+        assert res[act][0] == 0.0
+    # sigma(ln 3) = 3/4, so silu(ln 3) = 0.75 ln 3; the fp32 argument is off ln 3 by dx ~ 1e-8, corrected
+    # to first order with silu'(ln 3) = 3/4 + ln 3 * 3/16
+    l3 = math.log(3.0)
+    assert abs(res["silu"][3] - (0.75 * l3 + (0.75 + l3 * 0.1875) * (v[3] - l3))) <= 1e-14
+    assert abs(res["gelu"][1] - 0.8413447460685429) <= 1e-15  # Phi(1), standard normal table
+
+
+def test_lcb_block_layernorm_row_moments(oracle_mod):
+    x = _blk(15, norm="layernorm", act="none", d=32)
+    x.epi_r.gamma = x.epi_c.gamma = None
+    x.epi_r.beta = x.epi_c.beta = None
+    yr, yc = _blk_run(oracle_mod, x)
+    for y in (yr, yc):
+        assert np.max(np.abs(y.mean(-1))) <= 1e-13
+        v = y.var(-1)
+        assert np.all(v <= 1.0) and np.all(v > 0.99)  # var/(var+eps) with var = O(1), eps = 1e-5
+
+
+def test_lcb_block_isolation_bitwise(oracle_mod):
+    x = _blk(16)
+    yr, _ = _blk_run(oracle_mod, x)
+    x2 = _blk(16)
+    x2.lcb.x_cand[...] = ri.normal(99, 1, x2.lcb.x_cand.shape)
+    x2.epi_c.residual[...] = ri.normal(99, 2, x2.epi_c.residual.shape)
+    x2.epi_c.gamma[...] = 3.0
+    yr2, _ = _blk_run(oracle_mod, x2)
+    assert np.array_equal(yr, yr2)
