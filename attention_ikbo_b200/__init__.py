@@ -9,6 +9,8 @@ functions raises.
 Operations ("ROCS: Request-Oriented Compute Sharing ...", arXiv:2607.27744):
   * :func:`rocs_lcb_forward` -- section 3.1.2 Eq. (6) via the section 4.1 Eq. (14)
     decomposition, broadcast-add fused into the candidate GEMM epilogue (section 4.2).
+  * :func:`rocs_lcb_block_forward` -- the same with each output group's bias, residual,
+    group-local LayerNorm/RMSNorm and activation fused into the epilogue (section 3.1.3).
   * :func:`rocs_dca_forward` -- section 3.2 Eq. (13) candidate cross attention over K/V
     stored once per request (section 4.3).
   * :func:`rocs_dca_block_forward` -- both query groups of Eq. (13) with the K/V projections
@@ -27,6 +29,7 @@ from ._binding import (  # noqa: F401
     rocs_dca_block_forward,
     rocs_dca_forward,
     rocs_dca_forward_expand,
+    rocs_lcb_block_forward,
     rocs_lcb_forward,
     rocs_lcb_forward_expand,
     rocs_lcb_forward_fault_injection,

@@ -30,6 +30,15 @@ class LcbArgs(ctypes.Structure):
                 ("workspace", _vp), ("workspace_bytes", _sz)]
 
 
+class LcbEpilogue(ctypes.Structure):
+    _fields_ = [("bias", _vp), ("residual", _vp), ("gamma", _vp), ("beta", _vp), ("eps", _f32),
+                ("norm", _i32), ("act", _i32)]
+
+
+NORMS = {"none": 0, "layernorm": 1, "rmsnorm": 2}
+ACTS = {"none": 0, "relu": 1, "silu": 2, "gelu": 3}
+
+
 class DcaArgs(ctypes.Structure):
     _fields_ = [("R", _i64), ("q", _i64), ("H", _i64), ("dh", _i64), ("scale", _f32),
                 ("cand_off_dev", _vp), ("cand_off_host", _vp), ("seq_off_dev", _vp), ("seq_off_host", _vp),
@@ -73,6 +82,7 @@ def load_library():
             getattr(lib, name).argtypes = argt
         for name, argt in [("rocs_lcb_forward", [P(LcbArgs), _vp]), ("rocs_lcb_forward_expand", [P(LcbArgs), _vp]),
                            ("rocs_lcb_forward_noalloc", [P(LcbArgs), _vp]),
+                           ("rocs_lcb_block_forward", [P(LcbArgs), P(LcbEpilogue), P(LcbEpilogue), _vp]),
                            ("rocs_lcb_forward_fault_injection", [P(LcbArgs), _vp, _i64, _i64]),
                            ("rocs_dca_forward", [P(DcaArgs), _vp]), ("rocs_proj_forward", [P(ProjArgs), _vp]),
                            ("rocs_dca_forward_expand", [P(DcaArgs), _i64, _vp]),
@@ -202,6 +212,50 @@ def rocs_lcb_forward_fault_injection(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, 
     _check(lib.rocs_lcb_forward_fault_injection(ctypes.byref(a), _stream(stream), int(skip_release_request),
                                                 int(wait_limit_ns)), "rocs_lcb_forward_fault_injection")
     return ws
+
+
+def _epilogue(e, y_shape, dev, keep):
+    """``e``: dict with optional bias [o] / gamma [d] / beta [d] (fp32), residual (bf16, output shape),
+    eps, norm ("none" | "layernorm" | "rmsnorm"), act ("none" | "relu" | "silu" | "gelu"); or None."""
+    if e is None:
+        return None
+    def t(name, dtype, shape=None):
+        v = e.get(name)
+        if v is None:
+            return None
+        if not (isinstance(v, torch.Tensor) and v.is_cuda and v.is_contiguous() and v.dtype == dtype):
+            raise RocsError(1, f"epilogue {name} must be a contiguous CUDA {dtype} tensor")
+        if shape is not None and tuple(v.shape) != tuple(shape):
+            raise RocsError(1, f"epilogue {name} has shape {tuple(v.shape)}, expected {tuple(shape)}")
+        keep.append(v)
+        return v.data_ptr()
+    norm, act = e.get("norm", "none"), e.get("act", "none")
+    return LcbEpilogue(bias=t("bias", torch.float32, (y_shape[1],)),
+                       residual=t("residual", torch.bfloat16, y_shape),
+                       gamma=t("gamma", torch.float32, (y_shape[2],)), beta=t("beta", torch.float32, (y_shape[2],)),
+                       eps=float(e.get("eps", 1e-5)), norm=NORMS[norm] if isinstance(norm, str) else int(norm),
+                       act=ACTS[act] if isinstance(act, str) else int(act))
+
+
+def rocs_lcb_block_forward(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, epi_req=None, epi_cand=None, y_req=None,
+                           y_cand=None, workspace=None, stream=None):
+    """LCB block: IKBO-LCB with each group's bias / residual / norm / activation fused into the epilogue.
+
+    ``epi_req`` / ``epi_cand``: see :func:`_epilogue`.  Returns ``(y_req, y_cand)``.
+    """
+    lib = load_library()
+    a, keep, y_req, y_cand = _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y_cand)
+    hold = []
+    er = _epilogue(epi_req, tuple(y_req.shape), x_req.device, hold)
+    ec = _epilogue(epi_cand, tuple(y_cand.shape), x_req.device, hold)
+    nbytes = lib.rocs_lcb_workspace_size(ctypes.byref(a))
+    ws = _workspace(nbytes, x_req.device, workspace)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check(lib.rocs_lcb_block_forward(ctypes.byref(a), None if er is None else ctypes.byref(er),
+                                      None if ec is None else ctypes.byref(ec), _stream(stream)),
+           "rocs_lcb_block_forward")
+    rocs_lcb_block_forward.last_workspace = ws
+    return y_req, y_cand
 
 
 def rocs_lcb_forward_expand(*args, **kw):

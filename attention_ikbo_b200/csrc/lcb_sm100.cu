@@ -24,22 +24,34 @@
 // Tile shapes: M = 128 output rows (o_c, or a 128-row slice of o_r), N = d, K = n_c for a
 // candidate tile (K-blocks of 64 for request tiles, K = n_r).  A = weights (K-major),
 // B = embeddings X [K rows x d] (MN-major, d contiguous), both 128-byte swizzled.
+#include <type_traits>
+
 #include "lcb_sm100.h"
 
 namespace rocs {
 
 namespace {
 
-constexpr int kEpiWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kWarpsPerGroup = 4;  // one epilogue group covers the 128 TMEM lanes (tile rows)
 constexpr int kStages = 4;
+
+// NG epilogue groups of four warps, then the TMA producer warp and the tcgen05 issuer warp.
+// NG = 1: the group drains both TMEM accumulator buffers in turn; NG = 2: group g drains buffer g
+// only, so two tiles' epilogues run at once (used by the block epilogue, whose per-row work is long).
+template <int NG>
+struct LcbRoles {
+  static constexpr int kEpiWarps = kWarpsPerGroup * NG;
+  static constexpr int kProducerWarp = kEpiWarps;
+  static constexpr int kMmaWarp = kEpiWarps + 1;
+  static constexpr int kThreads = 32 * (kEpiWarps + 2);
+};
 constexpr uint32_t kSlot = 32768;  // one ring slot: a request k-block (A 16 KB + B <=16 KB) or one X^C tile
 constexpr int OC = 128;
 
-template <int D, int NC>
+template <int D, int NC, int NG>
 struct LcbSmem {
+  static constexpr int kEpiWarps = LcbRoles<NG>::kEpiWarps;
+  static constexpr int kStgPerWarp = 2 / NG;              // staging buffers per epilogue warp
   static constexpr uint32_t kWcc = NC * OC * 2;           // W_CC resident, NC/64 boxes of [128 x 64]
   static constexpr uint32_t kXc = NC * D * 2;             // one candidate's X^C tile
   static constexpr uint32_t kStgHalf = 32 * 128;          // 32 rows x 64 bf16 (one TMA store box)
@@ -47,26 +59,36 @@ struct LcbSmem {
   static constexpr uint32_t off_wcc = 0;
   static constexpr uint32_t off_ring = kWcc;
   static constexpr uint32_t off_stg = off_ring + kStages * kSlot;
-  static constexpr uint32_t off_bar = off_stg + kEpiWarps * 2 * kStgBuf;
-  static constexpr uint32_t n_bars = 2 * kStages + 2 + 2 + 2 + 2 + 1 + 1;
+  static constexpr uint32_t off_par = off_stg + kEpiWarps * kStgPerWarp * kStgBuf;
+  static constexpr uint32_t kPar = NG == 2 ? 2 * D * 4 : 0;  // block epilogue: candidate gamma, beta (fp32)
+  static constexpr uint32_t off_bar = off_par + kPar;
+  static constexpr uint32_t n_bars = 2 * kStages + 2 + 2 + 2 + 2 + 1 + 1 + kEpiWarps;
   static constexpr uint32_t off_misc = off_bar + n_bars * 8;
   static constexpr uint32_t bytes = off_misc + 64;
   static constexpr uint32_t alloc_bytes = bytes + 1024;  // slack for 1024-byte alignment
-  static constexpr uint32_t tmem_cols = (3 * D <= 256) ? 256 : 512;
+  static constexpr uint32_t tmem_cols = ((2 + NG) * D <= 256) ? 256 : 512;  // 2 accumulators + NG Z slots
+  static_assert((2 + NG) * D <= 512, "tensor memory budget");
   static_assert(kXc <= kSlot, "X^C tile must fit one slot");
   static_assert(alloc_bytes <= 232448, "shared memory budget");
 };
 
 }  // namespace
 
-template <int D, int NC>
-__global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __grid_constant__ LcbParams p) {
-  using L = LcbSmem<D, NC>;
+// EPI_C < 0: the plain LCB.  EPI_C >= 0: the LCB block epilogue, with the candidate group's
+// activation EPI_C fixed at compile time (the request group's is read at run time).
+template <int D, int NC, int EPI_C, int NG = EPI_C >= 0 ? 2 : 1>
+__global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kernel(const __grid_constant__ LcbParams p) {
+  using L = LcbSmem<D, NC, NG>;
+  constexpr bool EPI = EPI_C >= 0;
+  constexpr int kEpiWarps = LcbRoles<NG>::kEpiWarps;
+  constexpr int kProducerWarp = LcbRoles<NG>::kProducerWarp;
+  constexpr int kMmaWarp = LcbRoles<NG>::kMmaWarp;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_wcc = smem + L::off_wcc;
   uint8_t* s_ring = smem + L::off_ring;
   uint8_t* s_stg = smem + L::off_stg;
+  float* s_gb = reinterpret_cast<float*>(smem + L::off_par);  // block epilogue: gamma_C [D], beta_C [D]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
@@ -76,6 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
   uint64_t* wq_empty = wq_full + 2;
   uint64_t* wcc_bar = wq_empty + 2;
   uint64_t* drain_bar = wcc_bar + 1;
+  uint64_t* res_bar = drain_bar + 1;  // [kEpiWarps]: residual tile of each epilogue warp landed (block epilogue)
   int* s_wq = reinterpret_cast<int*>(smem + L::off_misc);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::off_misc + 16);
   int* s_abort = reinterpret_cast<int*>(smem + L::off_misc + 32);
@@ -98,18 +121,26 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&acc_full[k], 1);
-      mbar_init(&acc_empty[k], kEpiWarps);
+      mbar_init(&acc_empty[k], kWarpsPerGroup);  // the four warps of the group that drains buffer k
       mbar_init(&wq_full[k], 1);
       mbar_init(&wq_empty[k], 1 + kEpiWarps);
     }
     mbar_init(wcc_bar, 1);
     mbar_init(drain_bar, 1);
+    for (int k = 0; k < kEpiWarps; ++k) mbar_init(&res_bar[k], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
     tmem_alloc(s_tmem, L::tmem_cols);
     tmem_relinquish();
+  }
+  if constexpr (EPI) {
+    if (warp < kEpiWarps)
+      for (int k = threadIdx.x; k < D; k += 32 * kEpiWarps) {
+        s_gb[k] = p.epi_c.gamma ? p.epi_c.gamma[k] : 1.0f;
+        s_gb[D + k] = p.epi_c.beta ? p.epi_c.beta[k] : 0.0f;
+      }
   }
   tc_fence_before();
   __syncthreads();
@@ -215,13 +246,16 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
       mbar_drain(drain_bar, 0, 50000000ull);
     }
   } else {
-    // ------------------------------------------------------------------ epilogue warps 0..3
-    const int ew = warp;                       // owns TMEM lanes / tile rows 32*ew .. 32*ew+31
-    const uint32_t row = 32 * ew + lane;
-    const uint32_t t_lane = (uint32_t)(32 * ew) << 16;
-    const uint32_t z_tmem = tmem_base + t_lane + 2 * D;
-    uint32_t ab = 0, aph = 0, qs = 0, qph = 0, sb = 0;
+    // ------------------------------------------------------------------ epilogue warps
+    const int ew = warp;                 // epilogue warp index: staging buffers, residual barrier
+    const int quarter = warp & 3;        // owns TMEM lanes / tile rows 32*quarter .. 32*quarter+31
+    const int grp = warp >> 2;           // NG = 2: drains accumulator buffer grp only
+    const uint32_t row = 32 * quarter + lane;
+    const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
+    const uint32_t z_tmem = tmem_base + t_lane + (2 + grp) * D;  // this group's copy of Z_r
+    uint32_t ab = 0, aphs = 0, qs = 0, qph = 0, sb = 0;  // aphs bit b: phase of accumulator buffer b
     bool ok = true;
+    auto mine = [&]() { return NG == 1 || (int)ab == grp; };
 
     // write 32 accumulator columns (+ optional Z columns) of this thread's row as bf16 into the
     // warp's swizzled staging tile
@@ -244,20 +278,146 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
         bulk_commit();
       }
     };
-    auto acquire_stage = [&]() {  // staging buffer sb is free once the store issued two tiles ago has read it
-      if (lane == 0) bulk_wait_read<1>();
+    // block epilogue: fetch the residual rows of this warp's 32-row output tile into its staging
+    // buffer (same swizzled box as the store), add them, write the finished rows back in place
+    uint32_t rph = 0;
+    auto load_residual = [&](const CUtensorMap* tm, uint32_t stg_off, int y0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&res_bar[ew], (uint32_t)(D * 32 * 2));
+        for (int h = 0; h < D / 64; ++h) tma_load_2d(s_stg + stg_off + h * L::kStgHalf, tm, &res_bar[ew], h * 64, y0);
+      }
+    };
+    auto drain_residual = [&]() {  // a wait failed with a residual load possibly in flight
+      if (lane == 0) mbar_drain(&res_bar[ew], rph, 20000000ull);
       __syncwarp();
-      return (uint32_t)((ew * 2 + sb) * L::kStgBuf);
+    };
+    // One 64-column chunk of this thread's row (= one staging half) as 32 pairs: accumulator (+ Z)
+    // or + a per-row constant, + the residual from the staging buffer (loaded there in the store's
+    // swizzled layout).  Both 32-column TMEM loads (and both Z loads) are in flight before the wait.
+    auto load_chunk = [&](float2 (&xs)[32], uint32_t acc, bool use_z, float add, bool res, uint32_t stg, int c) {
+      if (use_z) {
+        uint32_t v0[32], v1[32], z0[32], z1[32];
+        tmem_ld32(acc + c * 64, v0);
+        tmem_ld32(z_tmem + c * 64, z0);
+        tmem_ld32(acc + c * 64 + 32, v1);
+        tmem_ld32(z_tmem + c * 64 + 32, z1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          xs[k] = __fadd2_rn(make_float2(__uint_as_float(v0[2 * k]), __uint_as_float(v0[2 * k + 1])),
+                             make_float2(__uint_as_float(z0[2 * k]), __uint_as_float(z0[2 * k + 1])));
+          xs[16 + k] = __fadd2_rn(make_float2(__uint_as_float(v1[2 * k]), __uint_as_float(v1[2 * k + 1])),
+                                  make_float2(__uint_as_float(z1[2 * k]), __uint_as_float(z1[2 * k + 1])));
+        }
+      } else {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(acc + c * 64, v0);
+        tmem_ld32(acc + c * 64 + 32, v1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          xs[k] = __fadd2_rn(make_float2(__uint_as_float(v0[2 * k]), __uint_as_float(v0[2 * k + 1])), f2(add));
+          xs[16 + k] = __fadd2_rn(make_float2(__uint_as_float(v1[2 * k]), __uint_as_float(v1[2 * k + 1])), f2(add));
+        }
+      }
+      if (res) {
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          const uint4 u = ld_shared_v4(stg + c * L::kStgHalf + lane * 128 + ((c16 ^ (lane & 7)) << 4));
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            xs[c16 * 4 + j] = __fadd2_rn(xs[c16 * 4 + j],
+                                         make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u)));
+        }
+      }
+    };
+    auto stage_chunk_f = [&](uint32_t stg, int c, const float2 (&xs)[32]) {
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16)
+        st_shared_v4(stg + c * L::kStgHalf + lane * 128 + ((c16 ^ (lane & 7)) << 4),
+                     pack_bf16x2(xs[c16 * 4].x, xs[c16 * 4].y), pack_bf16x2(xs[c16 * 4 + 1].x, xs[c16 * 4 + 1].y),
+                     pack_bf16x2(xs[c16 * 4 + 2].x, xs[c16 * 4 + 2].y),
+                     pack_bf16x2(xs[c16 * 4 + 3].x, xs[c16 * 4 + 3].y));
+    };
+    // The group's epilogue over the row.  With a norm: a statistics pass over the chunks that also
+    // writes acc (+ Z) (+ bias) (+ residual) back into the accumulator's TMEM columns, then an output
+    // pass that reads only those columns.  Without a norm: one pass.  No whole row is ever held in
+    // registers.  `act_ct` >= 0: activation fixed at compile time and gamma/beta from shared memory
+    // (the candidate group); < 0: e.act read at run time, gamma/beta from global memory.
+    auto epilogue_row = [&](auto act_ct, uint32_t acc, bool use_z, float add, bool res, uint32_t stg,
+                            const EpiGroup& e) {
+      constexpr int ACT = decltype(act_ct)::value;
+      if (e.norm != EPI_NORM_NONE) {
+        RowStats st{0.0f, 0.0f, 0.0f};
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          float2 xs[32];
+          load_chunk(xs, acc, use_z, add, res, stg, c);
+          stats_add_chunk(st, xs, e.norm);
+          uint32_t u0[32], u1[32];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            u0[2 * k] = __float_as_uint(xs[k].x);
+            u0[2 * k + 1] = __float_as_uint(xs[k].y);
+            u1[2 * k] = __float_as_uint(xs[16 + k].x);
+            u1[2 * k + 1] = __float_as_uint(xs[16 + k].y);
+          }
+          tmem_st32(acc + c * 64, u0);
+          tmem_st32(acc + c * 64 + 32, u1);
+        }
+        tmem_st_wait();
+        float mean, inv;
+        stats_finish(st, D, e, mean, inv);
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(acc + c * 64, v0);
+          tmem_ld32(acc + c * 64 + 32, v1);
+          tmem_ld_wait();
+          float2 xs[32];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            xs[k] = make_float2(__uint_as_float(v0[2 * k]), __uint_as_float(v0[2 * k + 1]));
+            xs[16 + k] = make_float2(__uint_as_float(v1[2 * k]), __uint_as_float(v1[2 * k + 1]));
+          }
+          if constexpr (ACT >= 0) {
+            norm_chunk_smem(xs, s_gb + c * 64, s_gb + D + c * 64, mean, inv);
+            act_chunk<ACT>(xs);
+          } else {
+            norm_chunk(xs, c * 64, mean, inv, e);
+            act_chunk_rt(e.act, xs);
+          }
+          stage_chunk_f(stg, c, xs);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
+          float2 xs[32];
+          load_chunk(xs, acc, use_z, add, res, stg, c);
+          if constexpr (ACT >= 0) act_chunk<ACT>(xs);
+          else act_chunk_rt(e.act, xs);
+          stage_chunk_f(stg, c, xs);
+        }
+      }
     };
 
-    for (;;) {  // request tiles
+    auto acquire_stage = [&]() {  // staging buffer sb is free once the store that last used it has read it
+      if (lane == 0) bulk_wait_read<L::kStgPerWarp - 1>();
+      __syncwarp();
+      return (uint32_t)((ew * L::kStgPerWarp + sb) * L::kStgBuf);
+    };
+    auto next_stage = [&]() { sb = (sb + 1) % L::kStgPerWarp; };
+
+    for (;;) {  // request tiles: every epilogue warp reads every item (each item occupies one buffer)
       if (!mbar_wait(&wq_full[qs], qph, ctl, 301)) { ok = false; break; }
       const int item = s_wq[qs];
       __syncwarp();
       if (lane == 0) mbar_arrive(&wq_empty[qs]);
       if (++qs == 2) { qs = 0; qph ^= 1; }
       if (item < 0) break;
-      if (!mbar_wait(&acc_full[ab], aph, ctl, 302)) { ok = false; break; }
+      if (!mine()) { ab ^= 1; continue; }
+      if (!mbar_wait(&acc_full[ab], (aphs >> ab) & 1, ctl, 302)) { ok = false; break; }
       tc_fence_after();
       const uint32_t acc = tmem_base + t_lane + ab * D;
       if (item < R) {
@@ -265,11 +425,17 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
         // of one 4-column group are 512 contiguous bytes (coalesced store here and load later).
         const int r = item;
         float* zr = p.zws + (size_t)r * OC * D;
+        // block epilogue: the candidate group's bias is folded into Z once per request
+        const float bz = (EPI && p.epi_c.bias) ? __ldg(p.epi_c.bias + row) : 0.0f;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t v[32];
           tmem_ld32(acc + cc * 32, v);
           tmem_ld_wait();
+          if constexpr (EPI) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) + bz);
+          }
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             st_global_v4(zr + ((size_t)(cc * 8 + j) * OC + row) * 4, v[4 * j], v[4 * j + 1], v[4 * j + 2],
@@ -280,9 +446,10 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
         if (lane == 0) {
           mbar_arrive(&acc_empty[ab]);
           __threadfence();
-          if (r != p.skip_release) red_release_gpu_add(&p.flags[r], 1);  // 4 warps x 1 = this request's Z is complete
+          // the four warps of this group x 1 = this request's Z is complete
+          if (r != p.skip_release) red_release_gpu_add(&p.flags[r], 1);
         }
-      } else {
+      } else if constexpr (!EPI) {
         const int u = item - R, r = u / mt_r, mt = u % mt_r;
         const uint32_t stg_off = acquire_stage();
         const uint32_t stg = smem_u32(s_stg + stg_off);
@@ -296,10 +463,29 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
-        store_tile(&p.tm_yr, stg_off, r * p.o_r + mt * OC + 32 * ew);
-        sb ^= 1;
+        store_tile(&p.tm_yr, stg_off, r * p.o_r + mt * OC + 32 * quarter);
+        next_stage();
+      } else {  // Y^R tile with the request group's epilogue
+        const int u = item - R, r = u / mt_r, mt = u % mt_r;
+        const int y0 = r * p.o_r + mt * OC + 32 * quarter;
+        const uint32_t stg_off = acquire_stage();
+        const uint32_t stg = smem_u32(s_stg + stg_off);
+        const bool res = p.epi_r.has_residual != 0;
+        if (res) {
+          load_residual(&p.tm_res_r, stg_off, y0);
+          if (!mbar_wait(&res_bar[ew], rph, ctl, 303)) { drain_residual(); ok = false; break; }
+          rph ^= 1;
+        }
+        const float br = p.epi_r.bias ? __ldg(p.epi_r.bias + mt * OC + row) : 0.0f;
+        epilogue_row(std::integral_constant<int, -1>{}, acc, false, br, res, stg, p.epi_r);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        store_tile(&p.tm_yr, stg_off, y0);
+        next_stage();
       }
-      if (++ab == 2) { ab = 0; aph ^= 1; }
+      aphs ^= 1u << ab;
+      ab ^= 1;
     }
 
     if (ok && cbeg < cend) {  // candidate tiles
@@ -316,8 +502,9 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
           next_off = p.cand_off[r + 1];
         }
         if (r >= R || r < 0) { ctl.fail(ROCS_ERR_DEVICE_INDEX, 310); ok = false; break; }
-        if (r != r_staged) {  // stage Z_r (this warp's 32 rows) into TMEM once per request
-          if (!wait_flag_geq(&p.flags[r], kEpiWarps, ctl, 311)) { ok = false; break; }
+        if (!mine()) { ab ^= 1; continue; }
+        if (r != r_staged) {  // stage Z_r (this warp's 32 rows) into this group's TMEM slot once per request
+          if (!wait_flag_geq(&p.flags[r], kWarpsPerGroup, ctl, 311)) { ok = false; break; }
           const float* zr = p.zws + (size_t)r * OC * D;
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -335,27 +522,56 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
           tmem_st_wait();
           r_staged = r;
         }
-        if (!mbar_wait(&acc_full[ab], aph, ctl, 312)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t acc = tmem_base + t_lane + ab * D;
-        const uint32_t stg_off = acquire_stage();
-        const uint32_t stg = smem_u32(s_stg + stg_off);
+        if constexpr (!EPI) {
+          if (!mbar_wait(&acc_full[ab], (aphs >> ab) & 1, ctl, 312)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t acc = tmem_base + t_lane + ab * D;
+          const uint32_t stg_off = acquire_stage();
+          const uint32_t stg = smem_u32(s_stg + stg_off);
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t v[32], z[32];
-          tmem_ld32(acc + cc * 32, v);
-          tmem_ld32(z_tmem + cc * 32, z);
-          tmem_ld_wait();
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t v[32], z[32];
+            tmem_ld32(acc + cc * 32, v);
+            tmem_ld32(z_tmem + cc * 32, z);
+            tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) + __uint_as_float(z[k]));
-          stage_chunk(stg, cc, v);
+            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) + __uint_as_float(z[k]));
+            stage_chunk(stg, cc, v);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          store_tile(&p.tm_yc, stg_off, i * OC + 32 * quarter);
+        } else {  // candidate group's epilogue: residual prefetched before the accumulator is ready
+          const uint32_t stg_off = acquire_stage();
+          const uint32_t stg = smem_u32(s_stg + stg_off);
+          const bool res = p.epi_c.has_residual != 0;
+          if (res) {
+            load_residual(&p.tm_res_c, stg_off, i * OC + 32 * quarter);
+            // this group's tile after next: start its residual rows towards L2 now
+            if (lane == 0 && i + 2 * NG < cend)
+              for (int h = 0; h < D / 64; ++h) tma_prefetch_l2_2d(&p.tm_res_c, h * 64, (i + 2 * NG) * OC + 32 * quarter);
+          }
+          if (!mbar_wait(&acc_full[ab], (aphs >> ab) & 1, ctl, 312)) {
+            if (res) drain_residual();
+            ok = false;
+            break;
+          }
+          if (res) {
+            if (!mbar_wait(&res_bar[ew], rph, ctl, 313)) { drain_residual(); ok = false; break; }
+            rph ^= 1;
+          }
+          tc_fence_after();
+          epilogue_row(std::integral_constant<int, EPI_C>{}, tmem_base + t_lane + ab * D, true, 0.0f, res, stg,
+                       p.epi_c);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          store_tile(&p.tm_yc, stg_off, i * OC + 32 * quarter);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[ab]);
-        store_tile(&p.tm_yc, stg_off, i * OC + 32 * ew);
-        sb ^= 1;
-        if (++ab == 2) { ab = 0; aph ^= 1; }
+        next_stage();
+        aphs ^= 1u << ab;
+        ab ^= 1;
       }
     }
     if (lane == 0) bulk_wait<0>();  // every TMA store of this warp has completed
@@ -371,26 +587,39 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_lcb_sm100_kernel(const __gri
 }
 
 // ------------------------------------------------------------------------------------ host
-template <int D, int NC>
+template <int D, int NC, int EPI_C>
 static cudaError_t launch_t(const LcbParams& p, int grid, cudaStream_t st) {
-  using L = LcbSmem<D, NC>;
-  auto k = rocs_lcb_sm100_kernel<D, NC>;
+  constexpr int NG = EPI_C >= 0 ? 2 : 1;
+  using L = LcbSmem<D, NC, NG>;
+  auto k = rocs_lcb_sm100_kernel<D, NC, EPI_C, NG>;
   static bool attr_set = false;  // per instantiation; harmless if two threads race
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::alloc_bytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k<<<grid, kThreads, L::alloc_bytes, st>>>(p);
+  k<<<grid, LcbRoles<NG>::kThreads, L::alloc_bytes, st>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_lcb_sm100(const LcbParams& p, int d, int n_c, int grid, cudaStream_t st) {
-  if (d == 128 && n_c == 64) return launch_t<128, 64>(p, grid, st);
-  if (d == 128 && n_c == 128) return launch_t<128, 128>(p, grid, st);
-  if (d == 64 && n_c == 64) return launch_t<64, 64>(p, grid, st);
-  if (d == 64 && n_c == 128) return launch_t<64, 128>(p, grid, st);
+template <int EPI_C>
+static cudaError_t launch_e(const LcbParams& p, int d, int n_c, int grid, cudaStream_t st) {
+  if (d == 128 && n_c == 64) return launch_t<128, 64, EPI_C>(p, grid, st);
+  if (d == 128 && n_c == 128) return launch_t<128, 128, EPI_C>(p, grid, st);
+  if (d == 64 && n_c == 64) return launch_t<64, 64, EPI_C>(p, grid, st);
+  if (d == 64 && n_c == 128) return launch_t<64, 128, EPI_C>(p, grid, st);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_lcb_sm100(const LcbParams& p, int d, int n_c, bool epilogue, int grid, cudaStream_t st) {
+  if (!epilogue) return launch_e<-1>(p, d, n_c, grid, st);
+  switch (p.epi_c.act) {
+    case EPI_ACT_NONE: return launch_e<EPI_ACT_NONE>(p, d, n_c, grid, st);
+    case EPI_ACT_RELU: return launch_e<EPI_ACT_RELU>(p, d, n_c, grid, st);
+    case EPI_ACT_SILU: return launch_e<EPI_ACT_SILU>(p, d, n_c, grid, st);
+    case EPI_ACT_GELU: return launch_e<EPI_ACT_GELU>(p, d, n_c, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace rocs

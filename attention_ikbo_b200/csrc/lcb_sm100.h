@@ -1,6 +1,6 @@
 // lcb_sm100.h -- launch parameters of the IKBO kernels (internal to the library).
 #pragma once
-#include "sm100.cuh"
+#include "epilogue.cuh"
 
 namespace rocs {
 
@@ -20,8 +20,12 @@ struct LcbParams {
   int R, C, n_r, o_r;
   long long wait_limit_ns;  // limit of every wait in the kernel
   int skip_release;         // fault injection: the Z tile of this request never releases its flag (-1: none)
+  // LCB block epilogue (used by the epilogue instantiation only)
+  CUtensorMap tm_res_r;     // residual of Y^R viewed as [R*o_r, d], box {64, 32} (loads)
+  CUtensorMap tm_res_c;     // residual of Y^C viewed as [C*o_c, d], box {64, 32} (loads)
+  EpiGroup epi_r, epi_c;
 };
-cudaError_t launch_lcb_sm100(const LcbParams& p, int d, int n_c, int grid, cudaStream_t st);
+cudaError_t launch_lcb_sm100(const LcbParams& p, int d, int n_c, bool epilogue, int grid, cudaStream_t st);
 
 // fp32 CUDA-core IKBO-LCB (two launches: request GEMM, then candidate GEMM + fused Z add).
 struct LcbF32Params {

@@ -2,6 +2,7 @@
 // validation, workspace layout, TMA tensor-map construction and kernel launches.
 // No entry point allocates or frees memory or synchronises a stream (except
 // rocs_read_status, whose job is to synchronise and read).
+#include <cmath>
 #include <cstring>
 
 #include "lcb_sm100.h"
@@ -114,7 +115,35 @@ int lcb_validate(const rocs_lcb_args* a, int64_t* C) {
 struct LcbOpts {
   long long wait_ns = kDefaultWaitLimitNs;
   int skip_release = -1;  // fault injection only
+  bool block = false;     // LCB block: fused per-group epilogue
+  const rocs_lcb_epilogue* epi_r = nullptr;
+  const rocs_lcb_epilogue* epi_c = nullptr;
 };
+
+int epi_validate(const rocs_lcb_epilogue* e) {
+  if (!e) return ROCS_OK;
+  if (e->norm < ROCS_NORM_NONE || e->norm > ROCS_NORM_RMS || e->act < ROCS_ACT_NONE || e->act > ROCS_ACT_GELU)
+    return ROCS_ERR_INVALID_ARG;
+  if (!(e->eps >= 0.0f) || !std::isfinite(e->eps)) return ROCS_ERR_INVALID_ARG;
+  if ((e->residual && !al16(e->residual)) || (e->gamma && !al16(e->gamma)) || (e->beta && !al16(e->beta)))
+    return ROCS_ERR_INVALID_ARG;  // residual by TMA, gamma/beta as float4
+  if (e->bias && (reinterpret_cast<uintptr_t>(e->bias) & 3u)) return ROCS_ERR_INVALID_ARG;
+  return ROCS_OK;
+}
+
+EpiGroup epi_group(const rocs_lcb_epilogue* e) {
+  EpiGroup g;
+  std::memset(&g, 0, sizeof(g));
+  if (!e) return g;
+  g.bias = e->bias;
+  g.gamma = e->gamma;
+  g.beta = e->beta;
+  g.eps = e->eps;
+  g.norm = e->norm;
+  g.act = e->act;
+  g.has_residual = e->residual != nullptr;
+  return g;
+}
 
 int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaStream_t st, int* launches,
             const LcbOpts& opts = LcbOpts()) {
@@ -162,6 +191,17 @@ int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaSt
   ok &= tmap_bf16(&p.tm_wrr, a->w_rr, a->n_r, a->o_r, a->n_r * 2, 64, 128);
   ok &= tmap_bf16(&p.tm_wcr, a->w_cr, a->n_r, a->o_c, a->n_r * 2, 64, 128);
   ok &= tmap_bf16(&p.tm_yr, a->y_req, d, (uint64_t)a->R * a->o_r, rb, 64, 32);
+  if (opts.block) {
+    p.epi_r = epi_group(opts.epi_r);
+    p.epi_c = epi_group(opts.epi_c);
+    // residual maps: the same boxes as the output stores (unused maps get any valid descriptor)
+    p.tm_res_r = p.tm_yr;
+    p.tm_res_c = p.tm_yr;
+    if (p.epi_r.has_residual)
+      ok &= tmap_bf16(&p.tm_res_r, opts.epi_r->residual, d, (uint64_t)a->R * a->o_r, rb, 64, 32);
+    if (p.epi_c.has_residual && C > 0)
+      ok &= tmap_bf16(&p.tm_res_c, opts.epi_c->residual, d, (uint64_t)C * a->o_c, rb, 64, 32);
+  }
   if (!ok) return ROCS_ERR_CUDA;
   p.cand_off = a->cand_off_dev;
   p.zws = reinterpret_cast<float*>(w + L.z);
@@ -177,7 +217,7 @@ int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaSt
   int64_t grid = C > n_req_tiles ? C : n_req_tiles;
   if (grid > sm_count()) grid = sm_count();
   if (grid < 1) grid = 1;
-  if (launch_lcb_sm100(p, (int)a->d, (int)a->n_c, (int)grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  if (launch_lcb_sm100(p, (int)a->d, (int)a->n_c, opts.block, (int)grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
   *launches = 1;
   return ROCS_OK;
 }
@@ -325,6 +365,26 @@ int rocs_lcb_forward_fault_injection(const rocs_lcb_args* a, rocs_stream_t strea
   LcbOpts o;
   o.wait_ns = wait_limit_ns;
   o.skip_release = (int)skip_release_request;
+  int launches = 0;
+  WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
+  rc = lcb_run(a, C, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream), &launches, o);
+  if (rc == ROCS_OK) g_last_launches = launches;
+  return rc;
+}
+
+int rocs_lcb_block_forward(const rocs_lcb_args* a, const rocs_lcb_epilogue* epi_req,
+                           const rocs_lcb_epilogue* epi_cand, rocs_stream_t stream) {
+  int64_t C = 0;
+  int rc = lcb_validate(a, &C);
+  if (rc) return rc;
+  if (a->dtype != ROCS_BF16) return ROCS_ERR_UNSUPPORTED;  // the epilogue lives in the bf16 kernel
+  if ((rc = epi_validate(epi_req)) || (rc = epi_validate(epi_cand))) return rc;
+  if (!a->workspace || a->workspace_bytes < lcb_bytes(a) || (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ROCS_ERR_WORKSPACE;
+  LcbOpts o;
+  o.block = true;
+  o.epi_r = epi_req;
+  o.epi_c = epi_cand;
   int launches = 0;
   WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
   rc = lcb_run(a, C, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream), &launches, o);

@@ -38,7 +38,7 @@ from attention_ikbo_b200 import accounting as acc  # noqa: E402
 METRIC = "IKBO LCB/DCA TFLOP/s & candidates/s at 1 B200; % of bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SRC = {"lcb": "attention_ikbo_b200/csrc/lcb_sm100.cu", "dca": "attention_ikbo_b200/csrc/dca_sm100.cu",
-              "proj": "attention_ikbo_b200/csrc/proj_sm100.cu"}
+              "proj": "attention_ikbo_b200/csrc/proj_sm100.cu", "lcb_block": "attention_ikbo_b200/csrc/lcb_sm100.cu"}
 
 
 # ----------------------------------------------------------------------------------- parts
@@ -110,6 +110,75 @@ class LcbPart(Part):
         sel = rs.choice(x.C, size=min(n, x.C), replace=False)
         t0 = time.perf_counter()
         oracle.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, sel_req=[], sel_cand=sel)
+        return time.perf_counter() - t0, len(sel) / x.C
+
+
+class LcbBlockPart(LcbPart):
+    """LCB block: the LCB with each group's bias / residual / LayerNorm / activation in the epilogue."""
+    kernel = "lcb_block"
+
+    def __init__(self, b: ri.LcbBlockInputs, name="lcb_block"):
+        super().__init__(b.lcb, name)
+        self.b = b
+
+    def _epi_bytes(self):
+        x, n = self.x, 0
+        for e, rows in ((self.b.epi_r, x.R * x.o_r), (self.b.epi_c, x.C * x.o_c)):
+            if e.residual is not None:
+                n += rows * x.d * 2
+            n += sum(a.size * 4 for a in (e.bias, e.gamma, e.beta) if a is not None)
+        return n
+
+    def bytes(self):
+        return acc.lcb_bytes(*self.dims()) + self._epi_bytes()
+
+    def _epi_dev(self, torch, e, dev):
+        out = {"eps": e.eps, "norm": e.norm, "act": e.act}
+        for k in ("bias", "gamma", "beta"):
+            if getattr(e, k) is not None:
+                out[k] = _to_dev(torch, getattr(e, k), dev)
+        return out
+
+    def to_device(self, ikbo, torch, dev):
+        x, b = self.x, self.b
+        self.h_in = [_pin(torch, a) for a in (x.x_req, x.x_cand)]
+        self.h_res = [_pin(torch, e.residual) for e in (b.epi_r, b.epi_c) if e.residual is not None]
+        self.d_in = [h.to(dev) for h in self.h_in]
+        self.d_res = [h.to(dev) for h in self.h_res]
+        self.d_w = [_to_dev(torch, a, dev) for a in (x.w_rr, x.w_cr, x.w_cc)]
+        self.epi = [self._epi_dev(torch, e, dev) for e in (b.epi_r, b.epi_c)]
+        k = 0
+        for e, de in zip((b.epi_r, b.epi_c), self.epi):
+            if e.residual is not None:
+                de["residual"] = self.d_res[k]
+                k += 1
+        self.off = ikbo.offsets(x.cand_off, dev)
+        self.h_off = _pin(torch, x.cand_off)
+        self.y_req = torch.empty((x.R, x.o_r, x.d), dtype=torch.bfloat16, device=dev)
+        self.y_cand = torch.empty((x.C, x.o_c, x.d), dtype=torch.bfloat16, device=dev)
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (self.y_req, self.y_cand)]
+        ikbo.rocs_lcb_block_forward(*self.d_in, *self.d_w, self.off, *self.epi, self.y_req, self.y_cand)
+        self.ws = ikbo.rocs_lcb_block_forward.last_workspace
+
+    def run(self, ikbo):
+        ikbo.rocs_lcb_block_forward(*self.d_in, *self.d_w, self.off, *self.epi, self.y_req, self.y_cand,
+                                    workspace=self.ws)
+        return ikbo.last_launch_count()
+
+    def h2d(self):
+        n = super().h2d()
+        for h, d in zip(self.h_res, self.d_res):
+            d.copy_(h, non_blocking=True)
+            n += h.numel() * h.element_size()
+        return n
+
+    def oracle_sample(self, oracle, n, seed):
+        x, b = self.x, self.b
+        rs = np.random.RandomState(seed)
+        sel = rs.choice(x.C, size=min(n, x.C), replace=False)
+        t0 = time.perf_counter()
+        oracle.lcb_block(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, b.epi_r, b.epi_c, sel_req=[],
+                         sel_cand=sel)
         return time.perf_counter() - t0, len(sel) / x.C
 
 
@@ -356,6 +425,8 @@ def make_parts(workload):
         return [DcaPart(ri.dca_bf16())]
     if workload == "dca_block":
         return [DcaBlockPart(ri.dca_block())]
+    if workload == "lcb_block":
+        return [LcbBlockPart(ri.lcb_block())]
     if workload == "chain":
         ci = ri.chain()
         lcb = LcbPart(ci.lcb, "chain_lcb")
@@ -376,7 +447,7 @@ def workload_config(workload, parts):
         x = p.x
         if isinstance(p, LcbPart):
             cfg["parts"][p.name] = {"R": x.R, "C": x.C, "n_r": x.n_r, "n_c": x.n_c, "d": x.d, "o_r": x.o_r,
-                                    "o_c": x.o_c, "recipe": x.recipe}
+                                    "o_c": x.o_c, "recipe": p.b.recipe if isinstance(p, LcbBlockPart) else x.recipe}
         elif isinstance(p, DcaBlockPart):
             cfg["parts"][p.name] = {"R": x.R, "C": x.C, "q": x.q, "q_req": x.q_req, "H": x.H, "dh": x.dh,
                                     "d_s": int(x.s_seq.shape[1]), "sum_L": int(x.seq_off[-1]), "recipe": x.recipe}
@@ -670,7 +741,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ikbo", choices=["ikbo", "reference"])
     ap.add_argument("--workload", default="ikbo_step",
-                    choices=["ikbo_step", "lcb", "dca", "dca_short", "dca_block", "chain"])
+                    choices=["ikbo_step", "lcb", "lcb_block", "dca", "dca_short", "dca_block", "chain"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--no-e2e", action="store_true")

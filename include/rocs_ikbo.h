@@ -153,6 +153,44 @@ ROCS_API int rocs_lcb_forward_fault_injection(const rocs_lcb_args* args, rocs_st
 ROCS_API int rocs_lcb_forward_noalloc(const rocs_lcb_args* args, rocs_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * LCB block: IKBO-LCB with a fused per-group output epilogue
+ *   (section 3.1.2 Eq. (4) bias; section 3.1.3 Eq. (7) group-local norm and Eq. (8)
+ *    pointwise merge / activation)
+ *
+ * For every output row y (length d) of group g in {R, C}, in this order:
+ *   y = (W X)_row + bias_g[o]                 o = the row's index within the group's o_g rows
+ *   y = y + residual_g[row]                    if residual_g != NULL
+ *   y = Norm_g(y) * gamma_g + beta_g           LayerNorm (population variance) or RMSNorm over
+ *                                              the row's d entries, eps_g inside the square root
+ *   y = act_g(y)                               ReLU, SiLU or GELU (erf form)
+ * Each group uses only its own parameters and its own rows, so the request outputs stay
+ * independent of the candidate inputs (Eq. (1)).  The candidate bias is folded into Z once
+ * per request (Eq. (14)); the norm's statistics stay in the thread that owns the row.
+ *
+ *   bias     [o_g] fp32, or NULL (0)      gamma, beta [d] fp32 16-byte aligned, or NULL (1, 0)
+ *   residual bf16, shape of the group's output ([R, o_r, d] or [C, o_c, d]), or NULL;
+ *            16-byte aligned (read by TMA)
+ *   norm     ROCS_NORM_*;  act ROCS_ACT_*;  eps >= 0 and finite
+ * dtype must be ROCS_BF16 (else ROCS_ERR_UNSUPPORTED); sizes, workspace and errors as for
+ * rocs_lcb_forward (workspace: rocs_lcb_workspace_size).  A NULL epilogue pointer means no
+ * epilogue for that group.  One kernel launch plus one memset.
+ * ---------------------------------------------------------------------------------- */
+typedef enum { ROCS_NORM_NONE = 0, ROCS_NORM_LAYER = 1, ROCS_NORM_RMS = 2 } rocs_norm;
+typedef enum { ROCS_ACT_NONE = 0, ROCS_ACT_RELU = 1, ROCS_ACT_SILU = 2, ROCS_ACT_GELU = 3 } rocs_act;
+typedef struct {
+  const float* bias;
+  const void* residual;
+  const float* gamma;
+  const float* beta;
+  float eps;
+  int32_t norm; /* rocs_norm */
+  int32_t act;  /* rocs_act */
+} rocs_lcb_epilogue;
+
+ROCS_API int rocs_lcb_block_forward(const rocs_lcb_args* args, const rocs_lcb_epilogue* epi_req,
+                                    const rocs_lcb_epilogue* epi_cand, rocs_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * IKBO-DCA  (section 3.2 Eq. (13); section 4.3)
  *
  *   q_ptr  [C*q, H, dh] bf16   query tokens; candidate i owns rows i*q .. i*q+q-1

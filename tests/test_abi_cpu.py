@@ -118,3 +118,23 @@ def test_fault_injection_host_validation(lib):
     assert lib.rocs_lcb_forward_fault_injection(ctypes.byref(a), None, 0, 10) == 1  # limit below 1 ms
     f32, keep2 = _lcb_args(m, [0, 3, 6], dtype=0, ws_bytes=1 << 20)
     assert lib.rocs_lcb_forward_fault_injection(ctypes.byref(f32), None, 0, 10_000_000) == 3
+
+
+def test_lcb_block_host_validation(lib):
+    import attention_ikbo_b200 as m
+
+    E = m._binding.LcbEpilogue
+    a, keep = _lcb_args(m, [0, 3, 6], ws_bytes=1 << 20)
+    P = ctypes.byref
+    assert lib.rocs_lcb_block_forward(P(a), P(E(norm=3)), None, None) == 1  # unknown norm
+    assert lib.rocs_lcb_block_forward(P(a), None, P(E(act=4)), None) == 1  # unknown activation
+    assert lib.rocs_lcb_block_forward(P(a), None, P(E(eps=-1.0)), None) == 1  # negative eps
+    assert lib.rocs_lcb_block_forward(P(a), None, P(E(eps=float("nan"))), None) == 1
+    assert lib.rocs_lcb_block_forward(P(a), None, P(E(residual=0x10008)), None) == 1  # TMA needs 16 B
+    assert lib.rocs_lcb_block_forward(P(a), P(E(bias=0x10002)), None, None) == 1  # fp32 alignment
+    f32, keep2 = _lcb_args(m, [0, 3, 6], dtype=0, ws_bytes=1 << 20)
+    assert lib.rocs_lcb_block_forward(P(f32), None, None, None) == 3  # bf16 kernel only
+    bad, keep3 = _lcb_args(m, [0, 3, 2], ws_bytes=1 << 20)
+    assert lib.rocs_lcb_block_forward(P(bad), None, None, None) == 2
+    small, keep4 = _lcb_args(m, [0, 3, 6], ws_bytes=100)
+    assert lib.rocs_lcb_block_forward(P(small), None, None, None) == 6
