@@ -19,6 +19,10 @@ paper-archivist reading notes:
 * :func:`lcb_block` -- section 3.1.2 Eq. (4)-(6) with section 3.1.3 Eq. (7)-(8): the LCB with a
   per-row bias, a residual merge, a group-local LayerNorm/RMSNorm over d and an activation, each
   output group with its own parameters (broadcast materialised as in :func:`lcb`).
+* :func:`fm` -- section 3.1.4, Eq. (9)-(10): the GLM-masked factorization machine, per candidate
+  the Gram matrix of the materialised [X^R; X^C] with the block mask, plus the request output.
+* :func:`pad_cols` / :func:`unpad_cols` -- the alignment transform of section 4.2.4 (zero padding of a
+  contiguous dimension), written as its definition.
 * :func:`proj` / :func:`chain` -- the chained block: LCB output -> bf16 -> linear
   query projection (section 3.2, Eq. (12), read as a plain linear map) -> bf16 -> DCA.
 
@@ -87,6 +91,7 @@ def _L():
                                               i64, vp, vp, vp, i64, vp, vp, vp, i32]
         lib.rocs_oracle_lcb_block.argtypes = [i64, vp, i64, i64, i64, i64, i64, vp, vp, vp, vp, vp,
                                               ctypes.POINTER(Epi), ctypes.POINTER(Epi), i64, vp, vp, i64, vp, vp, i32]
+        lib.rocs_oracle_fm.argtypes = [i64, vp, i64, i64, i64, vp, vp, i64, vp, vp, i64, vp, vp, i32]
         lib.rocs_oracle_round_bf16.restype = dbl
         lib.rocs_oracle_round_bf16.argtypes = [dbl]
         lib.rocs_oracle_max_threads.restype = i32
@@ -250,3 +255,34 @@ def lcb_block(cand_off, x_req, x_cand, w_rr, w_cr, w_cc, epi_r, epi_c, sel_req=N
     if rc != ORC_OK:
         raise OracleError(rc)
     return y_req, y_cand
+
+
+def fm(cand_off, x_req, x_cand, sel_req=None, sel_cand=None, nthreads: int = 0):
+    """Eq. (10).  Returns ``(y_req [n_sel_r, n_r, n_r], y_cand [n_sel_c, n_c, n_r + n_c])`` in float64."""
+    cand_off = _c(cand_off, np.int32)
+    R, C = len(cand_off) - 1, int(cand_off[-1])
+    _, n_r, d = x_req.shape
+    n_c = x_cand.shape[1]
+    sr = np.arange(R, dtype=np.int64) if sel_req is None else _c(sel_req, np.int64)
+    sc = np.arange(C, dtype=np.int64) if sel_cand is None else _c(sel_cand, np.int64)
+    y_req = np.empty((len(sr), n_r, n_r))
+    y_cand = np.empty((len(sc), n_c, n_r + n_c))
+    xr, xc = _c(x_req, np.uint16), _c(x_cand, np.uint16)
+    rc = _L().rocs_oracle_fm(R, _p(cand_off), n_r, n_c, d, _p(xr), _p(xc), len(sr), _p(sr), _p(y_req), len(sc),
+                             _p(sc), _p(y_cand), nthreads)
+    if rc != ORC_OK:
+        raise OracleError(rc)
+    return y_req, y_cand
+
+
+def pad_cols(a, cols_pad):
+    """Section 4.2.4: zero-pad the last (contiguous) axis of ``a`` to ``cols_pad`` entries."""
+    a = np.asarray(a)
+    out = np.zeros(a.shape[:-1] + (cols_pad,), dtype=a.dtype)
+    out[..., :a.shape[-1]] = a
+    return out
+
+
+def unpad_cols(a, cols):
+    """Inverse of :func:`pad_cols`: the first ``cols`` entries of the last axis."""
+    return np.ascontiguousarray(np.asarray(a)[..., :cols])

@@ -496,6 +496,67 @@ int rocs_oracle_lcb_block(int64_t R, const int32_t* cand_off, int64_t n_r, int64
   return bad ? ORC_ISOLATION : ORC_OK;
 }
 
+// GLM-masked factorization machine (section 3.1.4, Eq. (9)-(10)), bf16 inputs X^R [R, n_r, d],
+// X^C [C, n_c, d].  For every selected candidate the full input [X^R_{m_i}; X^C_i] is copied (the
+// materialised broadcast), its Gram matrix G = X_full X_full^T is formed in fp64, the block mask of
+// Eq. (9) is applied (output group R keeps only its interactions with group R: the R-rows' C-columns
+// are set to zero) and the candidate rows [n_r, n_r + n_c) are returned:
+//     Y^C_i = [X^C_i X^R_{m_i}^T , X^C_i X^C_i^T]          y_cand [n_sel_c, n_c, n_r + n_c]
+// Y^R_r = X^R_r X^R_r^T for the selected requests        y_req  [n_sel_r, n_r, n_r]
+// The masked R-rows of each candidate's full output must equal Y^R of its request computed alone and
+// hold exact zeros in the C-columns (Eq. (11)); otherwise ORC_ISOLATION.
+static void fm_request(const uint16_t* x_req, int64_t n_r, int64_t d, int64_t r, double* y) {
+  for (int64_t j = 0; j < n_r; ++j)
+    for (int64_t k = 0; k < n_r; ++k) {
+      double acc = 0.0;
+      for (int64_t c = 0; c < d; ++c) acc += widen(x_req, 1, (r * n_r + j) * d + c) * widen(x_req, 1, (r * n_r + k) * d + c);
+      y[j * n_r + k] = acc;
+    }
+}
+
+int rocs_oracle_fm(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n_c, int64_t d, const uint16_t* x_req,
+                   const uint16_t* x_cand, int64_t n_sel_r, const int64_t* sel_r, double* y_req, int64_t n_sel_c,
+                   const int64_t* sel_c, double* y_cand, int nthreads) {
+  if (n_r < 0 || n_c < 0 || d < 0) return ORC_INVALID;
+  if (!csr_ok(cand_off, R, -1)) return ORC_BAD_OFFSETS;
+  set_threads(nthreads);
+  const int64_t C = cand_off[R], n = n_r + n_c;
+  for (int64_t k = 0; k < n_sel_r; ++k)
+    if (sel_r[k] < 0 || sel_r[k] >= R) return ORC_INVALID;
+  for (int64_t k = 0; k < n_sel_c; ++k)
+    if (sel_c[k] < 0 || sel_c[k] >= C) return ORC_INVALID;
+  std::vector<int64_t> m = index_map(cand_off, R);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t k = 0; k < n_sel_r; ++k) fm_request(x_req, n_r, d, sel_r[k], y_req + k * n_r * n_r);
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t k = 0; k < n_sel_c; ++k) {
+    const int64_t i = sel_c[k], r = m[(size_t)i];
+    std::vector<double> X((size_t)(n * d)), G((size_t)(n * n));
+    for (int64_t j = 0; j < n_r; ++j)
+      for (int64_t c = 0; c < d; ++c) X[(size_t)(j * d + c)] = widen(x_req, 1, (r * n_r + j) * d + c);
+    for (int64_t j = 0; j < n_c; ++j)
+      for (int64_t c = 0; c < d; ++c) X[(size_t)((n_r + j) * d + c)] = widen(x_cand, 1, (i * n_c + j) * d + c);
+    for (int64_t a = 0; a < n; ++a)
+      for (int64_t b = 0; b < n; ++b) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c) acc += X[(size_t)(a * d + c)] * X[(size_t)(b * d + c)];
+        const bool masked = a < n_r && b >= n_r;  // M_{R,C} = 0 (Eq. 9)
+        G[(size_t)(a * n + b)] = masked ? 0.0 : acc;
+      }
+    std::vector<double> yr((size_t)(n_r * n_r));
+    fm_request(x_req, n_r, d, r, yr.data());
+    for (int64_t a = 0; a < n_r; ++a)
+      for (int64_t b = 0; b < n; ++b) {
+        const double want = b < n_r ? yr[(size_t)(a * n_r + b)] : 0.0;
+        if (G[(size_t)(a * n + b)] != want) bad |= 1;
+      }
+    for (int64_t a = 0; a < n_c; ++a)
+      for (int64_t b = 0; b < n; ++b) y_cand[(k * n_c + a) * n + b] = G[(size_t)((n_r + a) * n + b)];
+  }
+  return bad ? ORC_ISOLATION : ORC_OK;
+}
+
 // Exposed for the oracle's own tests of its bf16 rounding.
 double rocs_oracle_round_bf16(double x) { return round_bf16(x); }
 

@@ -544,3 +544,75 @@ def test_lcb_block_isolation_bitwise(oracle_mod):
     x2.epi_c.gamma[...] = 3.0
     yr2, _ = _blk_run(oracle_mod, x2)
     assert np.array_equal(yr, yr2)
+
+
+# ------------------------------------------------------------------------------ masked FM (f3)
+# Section 3.1.4 Eq. (9)-(10) and the alignment transform of section 4.2.4.
+def _fm_inputs(seed, counts=(2, 0, 3, 1), n_r=6, n_c=4, d=8):
+    return ri.make_lcb("t", list(counts), n_r, n_c, d, 8, 8, seed, "bf16")
+
+
+def test_fm_bruteforce_exact(oracle_mod):
+    x = _fm_inputs(21)
+    yr, yc = oracle_mod.fm(x.cand_off, x.x_req, x.x_cand)
+    xr = [[Fraction(float(v)) for v in row] for row in ri.bf16_to_f32(x.x_req).reshape(-1, x.d)]
+    xc = [[Fraction(float(v)) for v in row] for row in ri.bf16_to_f32(x.x_cand).reshape(-1, x.d)]
+    m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+    dot = lambda u, v: sum(a * b for a, b in zip(u, v))
+    for i in range(x.C):
+        rows_r = xr[m[i] * x.n_r:(m[i] + 1) * x.n_r]
+        for a in range(x.n_c):
+            u = xc[i * x.n_c + a]
+            want = [dot(u, v) for v in rows_r] + [dot(u, xc[i * x.n_c + b]) for b in range(x.n_c)]
+            assert [Fraction(float(v)) for v in yc[i, a]] == want
+    for r in range(x.R):
+        rows_r = xr[r * x.n_r:(r + 1) * x.n_r]
+        assert [[Fraction(float(v)) for v in row] for row in yr[r]] == [[dot(u, v) for v in rows_r] for u in rows_r]
+
+
+def test_fm_matches_library_and_symmetry(oracle_mod):
+    x = _fm_inputs(22, counts=(5, 3), n_r=16, n_c=8, d=32)
+    yr, yc = oracle_mod.fm(x.cand_off, x.x_req, x.x_cand)
+    xr = ri.bf16_to_f32(x.x_req).astype(np.float64)
+    xc = ri.bf16_to_f32(x.x_cand).astype(np.float64)
+    m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+    want_c = np.concatenate([np.einsum("iac,ibc->iab", xc, xr[m]), np.einsum("iac,ibc->iab", xc, xc)], axis=2)
+    assert np.max(np.abs(yc - want_c)) <= 1e-12 * np.max(np.abs(want_c))
+    assert np.max(np.abs(yr - np.einsum("rac,rbc->rab", xr, xr))) <= 1e-12 * np.max(np.abs(yr))
+    assert np.array_equal(yr, np.transpose(yr, (0, 2, 1)))
+    self_blk = yc[:, :, x.n_r:]
+    assert np.array_equal(self_blk, np.transpose(self_blk, (0, 2, 1)))
+
+
+def test_fm_closed_forms(oracle_mod):
+    # candidate embeddings equal to their request's: both blocks of Y^C equal Y^R of the request
+    x = _fm_inputs(23, counts=(2, 1, 2), n_r=5, n_c=5, d=8)
+    m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+    x.x_cand[...] = x.x_req[m]
+    yr, yc = oracle_mod.fm(x.cand_off, x.x_req, x.x_cand)
+    assert np.array_equal(yc[:, :, :5], yr[m]) and np.array_equal(yc[:, :, 5:], yr[m])
+    # zero candidate embeddings: Y^C = 0, Y^R unchanged
+    x.x_cand[...] = 0
+    yr2, yc2 = oracle_mod.fm(x.cand_off, x.x_req, x.x_cand)
+    assert np.array_equal(yr2, yr) and not np.any(yc2)
+
+
+def test_fm_isolation_bitwise(oracle_mod):
+    x = _fm_inputs(24)
+    yr, _ = oracle_mod.fm(x.cand_off, x.x_req, x.x_cand)
+    x.x_cand[...] = ri.normal(77, 1, x.x_cand.shape)
+    yr2, _ = oracle_mod.fm(x.cand_off, x.x_req, x.x_cand)
+    assert np.array_equal(yr, yr2)
+
+
+def test_pad_transform_leaves_the_computation_unchanged(oracle_mod):
+    # section 4.2.4: zero-pad the contiguous axis (30 -> 32 entries) and give the consumer's weight
+    # matching zero columns; the consumer's result is unchanged (small integers: exact)
+    rs = np.random.RandomState(5)
+    y = rs.randint(-4, 5, size=(7, 3, 30)).astype(np.float64)
+    w = rs.randint(-3, 4, size=(11, 3 * 30)).astype(np.float64)
+    yp = oracle_mod.pad_cols(y, 32)
+    assert yp.shape == (7, 3, 32) and not np.any(yp[..., 30:])
+    assert np.array_equal(oracle_mod.unpad_cols(yp, 30), y)
+    wp = oracle_mod.pad_cols(w.reshape(11, 3, 30), 32).reshape(11, 96)
+    assert np.array_equal(yp.reshape(7, 96) @ wp.T, y.reshape(7, 90) @ w.T)
