@@ -11,6 +11,9 @@ Operations ("ROCS: Request-Oriented Compute Sharing ...", arXiv:2607.27744):
     decomposition, broadcast-add fused into the candidate GEMM epilogue (section 4.2).
   * :func:`rocs_lcb_block_forward` -- the same with each output group's bias, residual,
     group-local LayerNorm/RMSNorm and activation fused into the epilogue (section 3.1.3).
+  * :func:`rocs_fm_forward` -- section 3.1.4 Eq. (10) masked FM with X^R kept on chip for all
+    candidates of a request, rows written in the aligned layout of section 4.2.4
+    (:func:`rocs_align_cols`, :func:`rocs_pad_cols`).
   * :func:`rocs_dca_forward` -- section 3.2 Eq. (13) candidate cross attention over K/V
     stored once per request (section 4.3).
   * :func:`rocs_dca_block_forward` -- both query groups of Eq. (13) with the K/V projections
@@ -26,14 +29,17 @@ from ._binding import (  # noqa: F401
     lib_path,
     load_library,
     offsets,
+    rocs_align_cols,
     rocs_dca_block_forward,
     rocs_dca_forward,
     rocs_dca_forward_expand,
+    rocs_fm_forward,
     rocs_lcb_block_forward,
     rocs_lcb_forward,
     rocs_lcb_forward_expand,
     rocs_lcb_forward_fault_injection,
     rocs_lcb_forward_noalloc,
+    rocs_pad_cols,
     rocs_proj_forward,
     rocs_read_status,
     STATUS_NAMES,

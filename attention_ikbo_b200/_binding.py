@@ -39,6 +39,12 @@ NORMS = {"none": 0, "layernorm": 1, "rmsnorm": 2}
 ACTS = {"none": 0, "relu": 1, "silu": 2, "gelu": 3}
 
 
+class FmArgs(ctypes.Structure):
+    _fields_ = [("R", _i64), ("n_r", _i64), ("n_c", _i64), ("d", _i64), ("cand_off_dev", _vp),
+                ("cand_off_host", _vp), ("x_req", _vp), ("x_cand", _vp), ("y_req", _vp), ("y_cand", _vp),
+                ("ld_req", _i64), ("ld_cand", _i64), ("workspace", _vp), ("workspace_bytes", _sz)]
+
+
 class DcaArgs(ctypes.Structure):
     _fields_ = [("R", _i64), ("q", _i64), ("H", _i64), ("dh", _i64), ("scale", _f32),
                 ("cand_off_dev", _vp), ("cand_off_host", _vp), ("seq_off_dev", _vp), ("seq_off_host", _vp),
@@ -77,7 +83,8 @@ def load_library():
         for name, argt in [("rocs_lcb_workspace_size", [P(LcbArgs)]), ("rocs_lcb_expand_workspace_size", [P(LcbArgs)]),
                            ("rocs_dca_workspace_size", [P(DcaArgs)]), ("rocs_proj_workspace_size", [P(ProjArgs)]),
                            ("rocs_dca_expand_workspace_size", [P(DcaArgs), _i64]),
-                           ("rocs_dca_block_workspace_size", [P(DcaBlockArgs)])]:
+                           ("rocs_dca_block_workspace_size", [P(DcaBlockArgs)]),
+                           ("rocs_fm_workspace_size", [P(FmArgs)])]:
             getattr(lib, name).restype = _sz
             getattr(lib, name).argtypes = argt
         for name, argt in [("rocs_lcb_forward", [P(LcbArgs), _vp]), ("rocs_lcb_forward_expand", [P(LcbArgs), _vp]),
@@ -87,9 +94,13 @@ def load_library():
                            ("rocs_dca_forward", [P(DcaArgs), _vp]), ("rocs_proj_forward", [P(ProjArgs), _vp]),
                            ("rocs_dca_forward_expand", [P(DcaArgs), _i64, _vp]),
                            ("rocs_dca_block_forward", [P(DcaBlockArgs), _vp]),
+                           ("rocs_fm_forward", [P(FmArgs), _vp]),
+                           ("rocs_pad_cols", [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _vp]),
                            ("rocs_read_status", [_vp, _vp, P(_i32), P(_i32)])]:
             getattr(lib, name).restype = ctypes.c_int
             getattr(lib, name).argtypes = argt
+        lib.rocs_align_cols.restype = _i64
+        lib.rocs_align_cols.argtypes = [_i64, _i64]
         lib.rocs_status_string.restype = ctypes.c_char_p
         lib.rocs_status_string.argtypes = [ctypes.c_int]
         lib.rocs_last_launch_count.restype = ctypes.c_int
@@ -391,3 +402,55 @@ def chain_forward(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, w_q, k_t, v_t, seq_
     o, lse = rocs_dca_forward(q.view(C, heads, head_dim), k_t, v_t, cand_off, seq_off, 1, scale,
                               workspace=ws.get("dca"), stream=stream)
     return y_req, y_cand, q, o, lse
+
+
+def rocs_align_cols(cols: int, elem_bytes: int) -> int:
+    """Smallest n >= cols with n * elem_bytes a multiple of 16 (section 4.2.4 alignment)."""
+    return int(load_library().rocs_align_cols(int(cols), int(elem_bytes)))
+
+
+def rocs_pad_cols(src, ld_dst, dst=None, stream=None):
+    """Copy the rows of ``src`` (last axis contiguous) into rows of ``ld_dst`` elements, zero-filling the
+    tail (section 4.2.4).  With ``ld_dst`` smaller than the source's last axis the rows are cut instead."""
+    lib = load_library()
+    if not (src.is_cuda and src.is_contiguous()):
+        raise RocsError(1, "rocs_pad_cols: src must be a contiguous CUDA tensor")
+    cols = min(src.shape[-1], ld_dst)
+    rows = src.numel() // src.shape[-1] if src.numel() else 0
+    if dst is None:
+        dst = torch.empty(tuple(src.shape[:-1]) + (ld_dst,), dtype=src.dtype, device=src.device)
+    _check(lib.rocs_pad_cols(_ptr(src), rows, cols, src.shape[-1], _ptr(dst), ld_dst, src.element_size(),
+                             _stream(stream)), "rocs_pad_cols")
+    return dst
+
+
+def rocs_fm_forward(x_req, x_cand, cand_off, y_req=None, y_cand=None, ld_req=0, ld_cand=0, workspace=None,
+                    stream=None):
+    """IKBO masked FM (Eq. 10).  Returns ``(y_req [R, n_r, ld_req], y_cand [C, n_c, ld_cand])``: the outputs
+    in their first n_r / n_r + n_c columns, zeros in the padding (ld 0 = the aligned default)."""
+    lib = load_library()
+    dev = x_req.device
+    off_d, off_h = _offsets(cand_off, dev)
+    R, n_r, d = x_req.shape
+    C = int(off_h[-1])
+    n_c = x_cand.shape[1]
+    ld_r = ld_req or rocs_align_cols(n_r, 2)
+    ld_c = ld_cand or rocs_align_cols(n_r + n_c, 2)
+    if y_req is None:
+        y_req = torch.empty((R, n_r, ld_r), dtype=torch.bfloat16, device=dev)
+    if y_cand is None:
+        y_cand = torch.empty((C, n_c, ld_c), dtype=torch.bfloat16, device=dev)
+    for t in (x_req, x_cand, y_req, y_cand):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16):
+            raise RocsError(1, "FM tensors must be contiguous CUDA bf16 tensors")
+    a = FmArgs(R=R, n_r=n_r, n_c=n_c, d=d, cand_off_dev=off_d.data_ptr(), cand_off_host=off_h.ctypes.data,
+               x_req=x_req.data_ptr(), x_cand=x_cand.data_ptr() if C else None, y_req=y_req.data_ptr(),
+               y_cand=y_cand.data_ptr() if C else None, ld_req=ld_r, ld_cand=ld_c)
+    nbytes = lib.rocs_fm_workspace_size(ctypes.byref(a))
+    if nbytes == 0:
+        _check(lib.rocs_fm_forward(ctypes.byref(a), _stream(stream)), "rocs_fm_forward")
+    ws = _workspace(nbytes, dev, workspace)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check(lib.rocs_fm_forward(ctypes.byref(a), _stream(stream)), "rocs_fm_forward")
+    rocs_fm_forward.last_workspace = ws
+    return y_req, y_cand

@@ -13,6 +13,10 @@ DCA (section 3.2 Eq. (13)):
   flops  4 * sum_r q N_r L_r H dh                      (S = Q K^T and O = P V)
   bytes  Q + K + V + O (+ LSE)
 Projection: flops 2 M N K, bytes in + W + out.
+Masked FM (section 3.1.4 Eq. (10)):
+  request part   2 n_r^2 d                             (X^R X^R^T once per request)
+  candidate part 2 n_c (n_r + n_c) d                   (cross block against the shared X^R, self block)
+  bytes          X^R, X^C, Y^R and Y^C at their unpadded row lengths (padding bytes are not counted)
 """
 from __future__ import annotations
 
@@ -56,3 +60,11 @@ def proj_flops(M, N, K):
 
 def proj_bytes(M, N, K, elem=2):
     return elem * (M * K + N * K + M * N)
+
+
+def fm_flops(R, C, n_r, n_c, d):
+    return R * 2 * n_r * n_r * d + C * 2 * n_c * (n_r + n_c) * d
+
+
+def fm_bytes(R, C, n_r, n_c, d, elem=2):
+    return elem * (R * n_r * d + C * n_c * d + R * n_r * n_r + C * n_c * (n_r + n_c))

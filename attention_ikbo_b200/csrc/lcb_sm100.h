@@ -75,6 +75,25 @@ struct ProjParams {
 };
 cudaError_t launch_proj_sm100(const ProjParams& p, int grid, cudaStream_t st);
 
+// IKBO masked factorization machine (bf16 in, fp32 accumulate, bf16 out in aligned rows).
+struct FmParams {
+  CUtensorMap tm_xr;   // X^R as [R][n_r][d], box {64, 128, 1}   (A of request tiles; rows past n_r read 0)
+  CUtensorMap tm_xrb;  // X^R as [R][n_r][d], box {64, n_b, 1}   (the resident B operand)
+  CUtensorMap tm_xc;   // X^C as [C*n_c, d],  box {64, 128}      (A of candidate tiles)
+  CUtensorMap tm_yr;   // Y^R as [R][n_r][ld_req], box {64, 32, 1} (stores)
+  CUtensorMap tm_yc;   // Y^C as [C*n_c, ld_cand], box {64, 32}   (stores)
+  const int32_t* cand_off;  // [R+1]
+  const int32_t* unit_off;  // [R+1], from the schedule kernel
+  WsHeader* ws;
+  int R, n_r, n_c, n_b, ld_req, ld_cand, n_units, req_tiles;
+  long long wait_limit_ns;
+};
+cudaError_t launch_fm_schedule(const int32_t* cand_off, int32_t* unit_off, int R, int n_c, int req_tiles,
+                               cudaStream_t st);
+cudaError_t launch_fm_sm100(const FmParams& p, int d, int grid, cudaStream_t st);
+cudaError_t launch_pad_cols(const void* in, int64_t rows, int64_t cols, int64_t ld_in, void* out, int64_t ld_out,
+                            int es, int grid, cudaStream_t st);
+
 // out[k] = k for k = 0..n (the identity candidate map: every request its own single candidate).
 cudaError_t launch_ident(int32_t* out, int n, cudaStream_t st);
 

@@ -57,6 +57,20 @@ bool tmap_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view [outer2][outer1][inner] with rows of row_bytes and planes of plane_bytes
+bool tmap_bf16_3d(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer1, uint64_t outer2,
+                  uint64_t row_bytes, uint64_t plane_bytes, uint32_t box_in, uint32_t box_1) {
+  EncodeTiledFn f = encode_fn();
+  if (!f || !base || inner == 0 || outer1 == 0 || outer2 == 0) return false;
+  cuuint64_t dims[3] = {inner, outer1, outer2};
+  cuuint64_t strides[2] = {row_bytes, plane_bytes};
+  cuuint32_t box[3] = {box_in, box_1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return f(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -522,6 +536,117 @@ extern "C" int rocs_dca_block_forward(const rocs_dca_block_args* a, rocs_stream_
   rc = dca_run(&d, a->R, L.T, L.units_r, hdr, w + L.body_r, st, &n, false);
   if (rc) return rc;
   g_last_launches = launches + n;
+  return ROCS_OK;
+}
+
+// ---------------------------------------------------------------- masked FM + alignment transform
+int64_t rocs_align_cols(int64_t cols, int64_t elem_bytes) {
+  if (cols < 0 || (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)) return -1;
+  const int64_t q = 16 / elem_bytes;  // elements per 16 bytes
+  return (cols + q - 1) / q * q;
+}
+
+int rocs_pad_cols(const void* src, int64_t rows, int64_t cols, int64_t ld_src, void* dst, int64_t ld_dst,
+                  int64_t elem_bytes, rocs_stream_t stream) {
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8) return ROCS_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0 || ld_src < cols || ld_dst < cols) return ROCS_ERR_INVALID_ARG;
+  if (rows == 0 || ld_dst == 0) return ROCS_OK;
+  if (!dst || (cols > 0 && !src)) return ROCS_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % (uintptr_t)elem_bytes)
+    return ROCS_ERR_INVALID_ARG;
+  const int64_t n = rows * ld_dst;
+  int64_t grid = (n + 255) / 256;
+  if (grid > 8 * sm_count()) grid = 8 * sm_count();
+  if (launch_pad_cols(src, rows, cols, ld_src, dst, ld_dst, (int)elem_bytes, (int)grid,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ROCS_ERR_CUDA;
+  g_last_launches = 1;
+  return ROCS_OK;
+}
+
+static int fm_validate(const rocs_fm_args* a, int64_t* C, int64_t* ld_r, int64_t* ld_c) {
+  if (!a) return ROCS_ERR_INVALID_ARG;
+  if (a->R < 0 || a->n_r <= 0 || a->n_c <= 0 || a->d <= 0) return ROCS_ERR_INVALID_ARG;
+  if ((a->d != 64 && a->d != 128) || (a->n_c != 32 && a->n_c != 64 && a->n_c != 128) || a->n_r > 256 || (a->n_r & 1))
+    return ROCS_ERR_UNSUPPORTED;
+  if (a->R > (1 << 28)) return ROCS_ERR_UNSUPPORTED;
+  int rc = check_csr(a->cand_off_host, a->R, C);
+  if (rc) return rc;
+  if (a->R > 0 && (!a->cand_off_dev || !a->x_req || !a->y_req)) return ROCS_ERR_INVALID_ARG;
+  if (*C > 0 && (!a->x_cand || !a->y_cand)) return ROCS_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->x_req, a->x_cand, a->y_req, a->y_cand};
+  for (const void* p : ptrs)
+    if (p && !al16(p)) return ROCS_ERR_INVALID_ARG;
+  *ld_r = a->ld_req ? a->ld_req : rocs_align_cols(a->n_r, 2);
+  *ld_c = a->ld_cand ? a->ld_cand : rocs_align_cols(a->n_r + a->n_c, 2);
+  if (*ld_r < a->n_r || *ld_c < a->n_r + a->n_c) return ROCS_ERR_INVALID_ARG;
+  if ((*ld_r * 2) % 16 || (*ld_c * 2) % 16 || *ld_r > 384 || *ld_c > 384) return ROCS_ERR_UNSUPPORTED;
+  if (*C * a->n_c >= (int64_t(1) << 31) || a->R * a->n_r >= (int64_t(1) << 31)) return ROCS_ERR_UNSUPPORTED;
+  return ROCS_OK;
+}
+
+static int64_t fm_units(const rocs_fm_args* a) {
+  const int64_t rt = (a->n_r + 127) / 128;
+  int64_t n = 0;
+  for (int64_t r = 0; r < a->R; ++r) n += rt + ((int64_t)(a->cand_off_host[r + 1] - a->cand_off_host[r]) * a->n_c + 127) / 128;
+  return n;
+}
+
+size_t rocs_fm_workspace_size(const rocs_fm_args* a) {
+  int64_t C, lr, lc;
+  if (fm_validate(a, &C, &lr, &lc) != ROCS_OK) return 0;
+  return sizeof(WsHeader) + a256((size_t)(a->R + 1) * sizeof(int32_t));
+}
+
+int rocs_fm_forward(const rocs_fm_args* a, rocs_stream_t stream) {
+  int64_t C = 0, ld_r = 0, ld_c = 0;
+  int rc = fm_validate(a, &C, &ld_r, &ld_c);
+  if (rc) return rc;
+  const size_t need = sizeof(WsHeader) + a256((size_t)(a->R + 1) * sizeof(int32_t));
+  if (!a->workspace || a->workspace_bytes < need || (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ROCS_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
+  int32_t* unit_off = reinterpret_cast<int32_t*>(hdr + 1);
+  if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return ROCS_ERR_CUDA;
+  if (a->R == 0) {
+    g_last_launches = 0;
+    return ROCS_OK;
+  }
+  const int64_t n_units = fm_units(a);
+  if (n_units >= (int64_t(1) << 31)) return ROCS_ERR_UNSUPPORTED;
+  const int rt = (int)((a->n_r + 127) / 128);
+  if (launch_fm_schedule(a->cand_off_dev, unit_off, (int)a->R, (int)a->n_c, rt, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  FmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint64_t d = a->d, n_r = a->n_r, R = a->R;
+  const uint32_t n_b = (uint32_t)((n_r + 15) / 16 * 16);
+  bool ok = tmap_bf16_3d(&p.tm_xr, a->x_req, d, n_r, R, d * 2, n_r * d * 2, 64, 128);
+  ok &= tmap_bf16_3d(&p.tm_xrb, a->x_req, d, n_r, R, d * 2, n_r * d * 2, 64, n_b);
+  ok &= tmap_bf16_3d(&p.tm_yr, a->y_req, (uint64_t)ld_r, n_r, R, (uint64_t)ld_r * 2, n_r * ld_r * 2, 64, 32);
+  if (C > 0) {
+    ok &= tmap_bf16(&p.tm_xc, a->x_cand, d, (uint64_t)C * a->n_c, d * 2, 64, 128);
+    ok &= tmap_bf16(&p.tm_yc, a->y_cand, (uint64_t)ld_c, (uint64_t)C * a->n_c, (uint64_t)ld_c * 2, 64, 32);
+  } else {  // no candidate tiles exist; any valid descriptor will do
+    p.tm_xc = p.tm_xr;
+    p.tm_yc = p.tm_yr;
+  }
+  if (!ok) return ROCS_ERR_CUDA;
+  p.cand_off = a->cand_off_dev;
+  p.unit_off = unit_off;
+  p.ws = hdr;
+  p.R = (int)R;
+  p.n_r = (int)n_r;
+  p.n_c = (int)a->n_c;
+  p.n_b = (int)n_b;
+  p.ld_req = (int)ld_r;
+  p.ld_cand = (int)ld_c;
+  p.n_units = (int)n_units;
+  p.req_tiles = rt;
+  p.wait_limit_ns = kDefaultWaitLimitNs;
+  int64_t grid = n_units < sm_count() ? n_units : sm_count();
+  if (launch_fm_sm100(p, (int)d, (int)grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  g_last_launches = 2;
   return ROCS_OK;
 }
 

@@ -38,7 +38,8 @@ from attention_ikbo_b200 import accounting as acc  # noqa: E402
 METRIC = "IKBO LCB/DCA TFLOP/s & candidates/s at 1 B200; % of bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SRC = {"lcb": "attention_ikbo_b200/csrc/lcb_sm100.cu", "dca": "attention_ikbo_b200/csrc/dca_sm100.cu",
-              "proj": "attention_ikbo_b200/csrc/proj_sm100.cu", "lcb_block": "attention_ikbo_b200/csrc/lcb_sm100.cu"}
+              "proj": "attention_ikbo_b200/csrc/proj_sm100.cu", "lcb_block": "attention_ikbo_b200/csrc/lcb_sm100.cu",
+              "fm": "attention_ikbo_b200/csrc/fm_sm100.cu"}
 
 
 # ----------------------------------------------------------------------------------- parts
@@ -179,6 +180,59 @@ class LcbBlockPart(LcbPart):
         t0 = time.perf_counter()
         oracle.lcb_block(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, b.epi_r, b.epi_c, sel_req=[],
                          sel_cand=sel)
+        return time.perf_counter() - t0, len(sel) / x.C
+
+
+class FmPart(Part):
+    """IKBO masked FM (Eq. 10), rows in the aligned (padded) layout."""
+    bound, kernel = "hbm", "fm"
+
+    def __init__(self, x: ri.FmInputs, name="fm"):
+        self.x, self.name = x, name
+        self.units = x.C
+
+    def flops(self):
+        x = self.x
+        return acc.fm_flops(x.R, x.C, x.n_r, x.n_c, x.d)
+
+    def bytes(self):
+        x = self.x
+        return acc.fm_bytes(x.R, x.C, x.n_r, x.n_c, x.d)
+
+    def to_device(self, ikbo, torch, dev):
+        x = self.x
+        self.h_in = [_pin(torch, a) for a in (x.x_req, x.x_cand)]
+        self.d_in = [h.to(dev) for h in self.h_in]
+        self.off = ikbo.offsets(x.cand_off, dev)
+        self.h_off = _pin(torch, x.cand_off)
+        self.y_req, self.y_cand = ikbo.rocs_fm_forward(*self.d_in, self.off)
+        self.ws = ikbo.rocs_fm_forward.last_workspace
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (self.y_req, self.y_cand)]
+
+    def run(self, ikbo):
+        ikbo.rocs_fm_forward(*self.d_in, self.off, self.y_req, self.y_cand, workspace=self.ws)
+        return ikbo.last_launch_count()
+
+    def h2d(self):
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+        self.off[0].copy_(self.h_off, non_blocking=True)
+        return sum(h.numel() * h.element_size() for h in self.h_in) + self.h_off.numel() * 4
+
+    def d2h(self):
+        for h, d in zip(self.h_out, (self.y_req, self.y_cand)):
+            h.copy_(d, non_blocking=True)
+        return sum(h.numel() * h.element_size() for h in self.h_out)
+
+    def status(self, ikbo):
+        return ikbo.rocs_read_status(self.ws)
+
+    def oracle_sample(self, oracle, n, seed):
+        x = self.x
+        rs = np.random.RandomState(seed)
+        sel = rs.choice(x.C, size=min(n, x.C), replace=False)
+        t0 = time.perf_counter()
+        oracle.fm(x.cand_off, x.x_req, x.x_cand, sel_req=[], sel_cand=sel)
         return time.perf_counter() - t0, len(sel) / x.C
 
 
@@ -427,6 +481,8 @@ def make_parts(workload):
         return [DcaBlockPart(ri.dca_block())]
     if workload == "lcb_block":
         return [LcbBlockPart(ri.lcb_block())]
+    if workload == "fm":
+        return [FmPart(ri.fm_bf16())]
     if workload == "chain":
         ci = ri.chain()
         lcb = LcbPart(ci.lcb, "chain_lcb")
@@ -448,6 +504,8 @@ def workload_config(workload, parts):
         if isinstance(p, LcbPart):
             cfg["parts"][p.name] = {"R": x.R, "C": x.C, "n_r": x.n_r, "n_c": x.n_c, "d": x.d, "o_r": x.o_r,
                                     "o_c": x.o_c, "recipe": p.b.recipe if isinstance(p, LcbBlockPart) else x.recipe}
+        elif isinstance(p, FmPart):
+            cfg["parts"][p.name] = {"R": x.R, "C": x.C, "n_r": x.n_r, "n_c": x.n_c, "d": x.d, "recipe": x.recipe}
         elif isinstance(p, DcaBlockPart):
             cfg["parts"][p.name] = {"R": x.R, "C": x.C, "q": x.q, "q_req": x.q_req, "H": x.H, "dh": x.dh,
                                     "d_s": int(x.s_seq.shape[1]), "sum_L": int(x.seq_off[-1]), "recipe": x.recipe}
@@ -741,7 +799,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ikbo", choices=["ikbo", "reference"])
     ap.add_argument("--workload", default="ikbo_step",
-                    choices=["ikbo_step", "lcb", "lcb_block", "dca", "dca_short", "dca_block", "chain"])
+                    choices=["ikbo_step", "lcb", "lcb_block", "fm", "dca", "dca_short", "dca_block", "chain"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--no-e2e", action="store_true")

@@ -191,6 +191,51 @@ ROCS_API int rocs_lcb_block_forward(const rocs_lcb_args* args, const rocs_lcb_ep
                                     const rocs_lcb_epilogue* epi_cand, rocs_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * IKBO masked factorization machine  (section 3.1.4 Eq. (9)-(10); section 4.1; section 4.2.4)
+ *
+ *   Y^R_r = X^R_r X^R_r^T                           once per request
+ *   Y^C_i = [ X^C_i X^R_{m_i}^T , X^C_i X^C_i^T ]    per candidate (n_r + n_c columns)
+ *
+ *   x_req  [R, n_r, d] bf16        x_cand [C, n_c, d] bf16        C = cand_off_host[R]
+ *   y_req  [R, n_r, ld_req] bf16   out: Y^R_r in columns [0, n_r), zeros in [n_r, ld_req)
+ *   y_cand [C, n_c, ld_cand] bf16  out: Y^C_i in columns [0, n_r + n_c), zeros beyond
+ * The leading dimensions are the alignment transform of section 4.2.4: 0 selects
+ * rocs_align_cols(n_r, 2) / rocs_align_cols(n_r + n_c, 2), the smallest row lengths whose byte
+ * size is a multiple of 16, so every row moves by TMA even when n_r + n_c alone would not; a
+ * consumer of the padded rows gives its weight zero columns at the padded positions (which
+ * rocs_pad_cols produces) and computes the same result.
+ * Supported: d in {64, 128}; n_c in {32, 64, 128}; n_r even and <= 256; ld_* multiples of 8 and
+ * <= 384; else ROCS_ERR_UNSUPPORTED.  Pointers 16-byte aligned.  fp32 accumulation, one bf16
+ * rounding per output.  Workspace: rocs_fm_workspace_size() bytes (status + a per-request tile
+ * table).  Two launches (tile table, FM kernel) plus one memset on `stream`.
+ * ---------------------------------------------------------------------------------- */
+typedef struct {
+  int64_t R, n_r, n_c, d;
+  const int32_t* cand_off_dev;  /* [R+1] */
+  const int32_t* cand_off_host; /* [R+1] */
+  const void* x_req;
+  const void* x_cand;
+  void* y_req;
+  void* y_cand;
+  int64_t ld_req, ld_cand; /* row lengths of y_req / y_cand in elements; 0 = aligned default */
+  void* workspace;
+  size_t workspace_bytes;
+} rocs_fm_args;
+
+ROCS_API size_t rocs_fm_workspace_size(const rocs_fm_args* args);
+ROCS_API int rocs_fm_forward(const rocs_fm_args* args, rocs_stream_t stream);
+
+/* Alignment transform helpers (section 4.2.4; no device memory of their own).
+ * rocs_align_cols: the smallest n >= cols with n * elem_bytes a multiple of 16 (elem_bytes in
+ *   {1, 2, 4, 8}; -1 otherwise).
+ * rocs_pad_cols: dst[r, 0:cols] = src[r, 0:cols], dst[r, cols:ld_dst] = 0 for r < rows, with row
+ *   strides ld_src / ld_dst in elements (ld_* >= cols).  With ld_dst == cols it removes padding.
+ *   Pointers aligned to elem_bytes; src and dst must not overlap.  One launch on `stream`. */
+ROCS_API int64_t rocs_align_cols(int64_t cols, int64_t elem_bytes);
+ROCS_API int rocs_pad_cols(const void* src, int64_t rows, int64_t cols, int64_t ld_src, void* dst, int64_t ld_dst,
+                           int64_t elem_bytes, rocs_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * IKBO-DCA  (section 3.2 Eq. (13); section 4.3)
  *
  *   q_ptr  [C*q, H, dh] bf16   query tokens; candidate i owns rows i*q .. i*q+q-1

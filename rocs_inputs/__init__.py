@@ -358,3 +358,42 @@ def lcb_block(seed: int = 7, R: int = 64, lo: int = 256, hi: int = 1024, residua
                 f"group, bias~N(0,0.25), {'residual~N(0,1) bf16, ' if residual else ''}LayerNorm over d "
                 f"(gamma~1+N(0,0.01), beta~N(0,0.01), eps 1e-5), SiLU; seed {seed}")
     return x
+
+
+# ---- masked FM (section 3.1.4, Eq. 10) -------------------------------------------------
+@dataclass
+class FmInputs:
+    name: str
+    cand_off: np.ndarray
+    n_r: int
+    n_c: int
+    d: int
+    x_req: np.ndarray  # uint16 [R, n_r, d]
+    x_cand: np.ndarray  # uint16 [C, n_c, d]
+    recipe: str = ""
+
+    @property
+    def R(self):
+        return len(self.cand_off) - 1
+
+    @property
+    def C(self):
+        return int(self.cand_off[-1])
+
+
+def make_fm(name, counts, n_r, n_c, d, seed, std=None) -> FmInputs:
+    """Embeddings ~ N(0, std^2) in bf16 (std = d^-1/4 keeps the Gram entries O(1))."""
+    off = counts_to_offsets(counts)
+    R, C = len(counts), int(off[-1])
+    s = float(std if std is not None else d ** -0.25)
+    return FmInputs(name=name, cand_off=off, n_r=n_r, n_c=n_c, d=d,
+                    x_req=normal(seed, S_XREQ, (R, n_r, d), s), x_cand=normal(seed, S_XCAND, (C, n_c, d), s))
+
+
+def fm_bf16(seed: int = 8, R: int = 64, lo: int = 256, hi: int = 1024, n_r: int = 250, n_c: int = 64,
+            d: int = 128) -> FmInputs:
+    counts = uniform_int(seed, S_NCAND, lo, hi, R)
+    x = make_fm("fm_bf16", counts, n_r, n_c, d, seed)
+    x.recipe = (f"R={R}, N_r~U{{{lo}..{hi}}}; n_r={n_r}, n_c={n_c}, d={d}; X~N(0, d^-1/2) bf16; output rows "
+                f"n_r+n_c={n_r + n_c} padded to 16-byte multiples; seed {seed}")
+    return x

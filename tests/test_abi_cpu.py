@@ -138,3 +138,35 @@ def test_lcb_block_host_validation(lib):
     assert lib.rocs_lcb_block_forward(P(bad), None, None, None) == 2
     small, keep4 = _lcb_args(m, [0, 3, 6], ws_bytes=100)
     assert lib.rocs_lcb_block_forward(P(small), None, None, None) == 6
+
+
+def test_fm_host_validation(lib):
+    import attention_ikbo_b200 as m
+
+    F = m._binding.FmArgs
+    fake = 0x10000
+
+    def args(off, n_r=64, n_c=64, d=128, ld_req=0, ld_cand=0, ws=1 << 20):
+        off = np.asarray(off, np.int32)
+        a = F(R=len(off) - 1, n_r=n_r, n_c=n_c, d=d, cand_off_dev=fake, cand_off_host=off.ctypes.data, x_req=fake,
+              x_cand=fake, y_req=fake, y_cand=fake, ld_req=ld_req, ld_cand=ld_cand, workspace=fake if ws else None,
+              workspace_bytes=ws)
+        return a, off
+
+    P = ctypes.byref
+    for kw, code in [({"d": 96}, 3), ({"n_c": 48}, 3), ({"n_r": 63}, 3), ({"n_r": 258}, 3),
+                     ({"ld_cand": 120}, 1), ({"ld_cand": 132}, 3), ({"ld_req": 60}, 1), ({"ld_cand": 392}, 3)]:
+        a, keep = args([0, 3, 5], **kw)
+        assert lib.rocs_fm_forward(P(a), None) == code, kw
+    a, keep = args([0, 3, 2])
+    assert lib.rocs_fm_forward(P(a), None) == 2
+    a, keep = args([0, 3, 5], ws=0)
+    assert lib.rocs_fm_forward(P(a), None) == 6
+    a, keep = args([0, 3, 5])
+    assert lib.rocs_fm_workspace_size(P(a)) == 256 + 256
+    assert lib.rocs_align_cols(314, 2) == 320 and lib.rocs_align_cols(320, 2) == 320
+    assert lib.rocs_align_cols(3, 8) == 4 and lib.rocs_align_cols(17, 1) == 32 and lib.rocs_align_cols(5, 3) == -1
+    assert lib.rocs_pad_cols(fake, 4, 10, 10, fake, 16, 3, None) == 1  # element size
+    assert lib.rocs_pad_cols(fake, 4, 10, 8, fake, 16, 2, None) == 1  # ld_src < cols
+    assert lib.rocs_pad_cols(fake + 1, 4, 10, 10, fake, 16, 2, None) == 1  # misaligned
+    assert lib.rocs_pad_cols(None, 0, 10, 10, None, 16, 2, None) == 0  # nothing to do
