@@ -16,6 +16,8 @@
 //
 // Roles: warps 0-3 epilogue (TMEM -> bf16 rows in the store's swizzled staging -> TMA stores), warp 4
 // TMA producer, warp 5 tcgen05 issuer.  TMEM: cross block [0, 256), self block [256, 384).
+#include <type_traits>
+
 #include "lcb_sm100.h"
 
 namespace rocs {
@@ -223,26 +225,51 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
     uint32_t aph = 0;
     // address of the 16-byte unit u (8 columns) of this lane's staging row (64-column TMA boxes,
     // 128-byte swizzle)
+    const uint32_t lane_base = stg_u + lane * 128, lx = lane & 7;
     auto unit_addr = [&](int u) -> uint32_t {
-      return stg_u + (uint32_t)(u >> 3) * (32 * 128) + lane * 128 + ((((uint32_t)u & 7) ^ (lane & 7)) << 4);
+      return lane_base + (uint32_t)(u >> 3) * (32 * 128) + ((((uint32_t)u & 7) ^ lx) << 4);
     };
-    // output columns [col0, col0 + cnt) of this lane's row from 32 fp32 values (cnt <= 32, col0 even)
-    auto put = [&](int col0, const uint32_t (&v)[32], int cnt) {
-      uint32_t pk[16];
+    auto pack = [&](const uint32_t (&v)[32], uint32_t (&pk)[16]) {
 #pragma unroll
       for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-      if ((col0 & 7) == 0 && cnt == 32) {
+    };
+    // output columns [col0, col0 + cnt) from 32 values, col0 a multiple of 8, cnt even
+    auto put_aligned = [&](int col0, const uint32_t (&v)[32], int cnt) {
+      uint32_t pk[16];
+      pack(v, pk);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          st_shared_v4(unit_addr((col0 >> 3) + j), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      for (int j = 0; j < 4; ++j)
+        if (8 * j + 8 <= cnt) st_shared_v4(unit_addr((col0 >> 3) + j), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        if (2 * k >= (cnt & ~7) && 2 * k < cnt) st_shared_u32(unit_addr((col0 >> 3) + (k >> 2)) + (k & 3) * 4, pk[k]);
+    };
+    // 32 output columns starting at col0 with col0 % 8 == S (S even, fixed at compile time): a
+    // partial unit of (8 - S) / 2 pairs, three whole units, a partial unit of S / 2 pairs
+    auto put_shifted = [&](auto s_ct, int col0, const uint32_t (&v)[32]) {
+      constexpr int S = decltype(s_ct)::value;
+      uint32_t pk[16];
+      pack(v, pk);
+      const int u0 = col0 >> 3;
+      if constexpr (S == 0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st_shared_v4(unit_addr(u0 + j), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
       } else {
+        constexpr int h = (8 - S) / 2;  // pairs in the first partial unit
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-          if (2 * k < cnt) {
-            const int c = col0 + 2 * k;
-            st_shared_u32(unit_addr(c >> 3) + (uint32_t)((c & 7) * 2), pk[k]);
-          }
+        for (int k = 0; k < h; ++k) st_shared_u32(unit_addr(u0) + S * 2 + 4 * k, pk[k]);
+#pragma unroll
+        for (int j = 0; j < 3; ++j)
+          st_shared_v4(unit_addr(u0 + 1 + j), pk[h + 4 * j], pk[h + 4 * j + 1], pk[h + 4 * j + 2], pk[h + 4 * j + 3]);
+#pragma unroll
+        for (int k = 0; k < S / 2; ++k) st_shared_u32(unit_addr(u0 + 4) + 4 * k, pk[h + 12 + k]);
       }
+    };
+    // 64 columns (two 32-column loads in flight) per TMEM round trip
+    auto load64 = [&](uint32_t taddr, uint32_t (&v)[2][32], bool second) {
+      tmem_ld32(taddr, v[0]);
+      if (second) tmem_ld32(taddr + 32, v[1]);
+      tmem_ld_wait();
     };
     for (int u = ubeg; u < uend; ++u) {
       unit_walk_advance(w, p.unit_off, R, u);
@@ -259,20 +286,29 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
         __syncwarp();
         for (int uu = ncols >> 3; uu < nbox * 8; ++uu) st_shared_v4(unit_addr(uu), 0u, 0u, 0u, 0u);  // pad
 #pragma unroll 1
-        for (int c = 0; c * 32 < n_r; ++c) {  // cross block (columns past n_r are the zero rows of B)
-          uint32_t v[32];
-          tmem_ld32(tmem_base + t_lane + c * 32, v);
-          tmem_ld_wait();
-          put(c * 32, v, min(32, n_r - c * 32));
+        for (int h = 0; 64 * h < n_r; ++h) {  // cross block (columns past n_r are the zero rows of B)
+          uint32_t v[2][32];
+          const int ch = n_r - 64 * h;
+          load64(tmem_base + t_lane + 64 * h, v, ch > 32);
+          put_aligned(64 * h, v[0], min(32, ch));
+          if (ch > 32) put_aligned(64 * h + 32, v[1], min(32, ch - 32));
         }
         if (cand) {  // self block: the n_c Gram columns of this row's own candidate
-          const int cb = (32 * q / n_c) * n_c;
+          const int cb = (32 * q / n_c) * n_c, sh = n_r & 7;
 #pragma unroll 1
-          for (int c = 0; c * 32 < n_c; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tmem_base + t_lane + 256 + cb + c * 32, v);
-            tmem_ld_wait();
-            put(n_r + c * 32, v, 32);
+          for (int h = 0; 64 * h < n_c; ++h) {
+            uint32_t v[2][32];
+            const bool two = n_c - 64 * h > 32;
+            load64(tmem_base + t_lane + 256 + cb + 64 * h, v, two);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              if (c == 1 && !two) break;
+              const int col0 = n_r + 64 * h + 32 * c;
+              if (sh == 0) put_shifted(std::integral_constant<int, 0>{}, col0, v[c]);
+              else if (sh == 2) put_shifted(std::integral_constant<int, 2>{}, col0, v[c]);
+              else if (sh == 4) put_shifted(std::integral_constant<int, 4>{}, col0, v[c]);
+              else put_shifted(std::integral_constant<int, 6>{}, col0, v[c]);
+            }
           }
         }
       }
