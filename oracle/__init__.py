@@ -23,6 +23,8 @@ paper-archivist reading notes:
   the Gram matrix of the materialised [X^R; X^C] with the block mask, plus the request output.
 * :func:`pad_cols` / :func:`unpad_cols` -- the alignment transform of section 4.2.4 (zero padding of a
   contiguous dimension), written as its definition.
+* :func:`chain_fold` -- the projection weight composed with W_CC (linear maps compose), used by the
+  chain that splits the projection over the IKBO decomposition.
 * :func:`proj` / :func:`chain` -- the chained block: LCB output -> bf16 -> linear
   query projection (section 3.2, Eq. (12), read as a plain linear map) -> bf16 -> DCA.
 
@@ -87,6 +89,8 @@ def _L():
         lib.rocs_oracle_proj.argtypes = [i64, i64, i64, vp, vp, vp, i32]
         lib.rocs_oracle_chain.argtypes = [i64, vp, i64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp,
                                           i64, i64, dbl, vp, vp, i64, vp, vp, vp, vp, vp, i32]
+        lib.rocs_oracle_chain_exact.argtypes = lib.rocs_oracle_chain.argtypes
+        lib.rocs_oracle_chain_fold.argtypes = [i64, i64, i64, i64, vp, vp, vp, i32]
         lib.rocs_oracle_dca_block.argtypes = [i64, vp, vp, i64, i64, i64, i64, i64, dbl, vp, vp, vp, vp, vp, vp, vp,
                                               i64, vp, vp, vp, i64, vp, vp, vp, i32]
         lib.rocs_oracle_lcb_block.argtypes = [i64, vp, i64, i64, i64, i64, i64, vp, vp, vp, vp, vp,
@@ -177,9 +181,11 @@ def proj(y_bf16, w_q, nthreads: int = 0):
     return out
 
 
-def chain(ci, sel_cand, nthreads: int = 0):
+def chain(ci, sel_cand, nthreads: int = 0, round_y: bool = True):
     """Chained block for candidates ``sel_cand`` of a ``rocs_inputs.ChainInputs``.
 
+    ``round_y``: Y^C is stored in bf16 between the LCB and the projection (the unfused chain); False:
+    the projection consumes the exact LCB output (the chain that never stores Y^C).
     Returns ``(y_cand [n,o_c,d], q [n,H*dh], o [n,H,dh], lse [n,H])`` in float64.
     """
     x = ci.lcb
@@ -190,7 +196,8 @@ def chain(ci, sel_cand, nthreads: int = 0):
     o = np.empty((n, ci.H, ci.dh), dtype=np.float64)
     lse = np.empty((n, ci.H), dtype=np.float64)
     co, so = _c(x.cand_off, np.int32), _c(ci.seq_off, np.int32)
-    rc = _L().rocs_oracle_chain(x.R, _p(co), x.n_r, x.n_c, x.d, x.o_r, x.o_c, _p(x.x_req), _p(x.x_cand),
+    fn = _L().rocs_oracle_chain if round_y else _L().rocs_oracle_chain_exact
+    rc = fn(x.R, _p(co), x.n_r, x.n_c, x.d, x.o_r, x.o_c, _p(x.x_req), _p(x.x_cand),
                                 _p(x.w_rr), _p(x.w_cr), _p(x.w_cc), _p(ci.w_q), _p(so), ci.H, ci.dh,
                                 float(ci.scale), _p(ci.k_t), _p(ci.v_t), n, _p(sel), _p(y), _p(qo), _p(o),
                                 _p(lse), nthreads)
@@ -286,3 +293,14 @@ def pad_cols(a, cols_pad):
 def unpad_cols(a, cols):
     """Inverse of :func:`pad_cols`: the first ``cols`` entries of the last axis."""
     return np.ascontiguousarray(np.asarray(a)[..., :cols])
+
+
+def chain_fold(w_q, w_cc, d: int, nthreads: int = 0):
+    """``W_fold[k, n*d + c] = sum_o W_q[k, o*d + c] W_CC[o, n]`` in float64 (bf16 inputs)."""
+    wq, wc = _c(w_q, np.uint16), _c(w_cc, np.uint16)
+    n_out, o_c, n_c = wq.shape[0], wc.shape[0], wc.shape[1]
+    out = np.empty((n_out, n_c * d))
+    rc = _L().rocs_oracle_chain_fold(n_out, o_c, n_c, d, _p(wq), _p(wc), _p(out), nthreads)
+    if rc != ORC_OK:
+        raise OracleError(rc)
+    return out

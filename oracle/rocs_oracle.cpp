@@ -347,15 +347,18 @@ int rocs_oracle_proj(int64_t n_rows, int64_t n_in, int64_t n_out, const uint16_t
 }
 
 // Chained block for the candidates in sel_cand (q = 1 query token per candidate):
-//   Y^C_i (LCB, Eq. 6) -> round to bf16 -> Q_i = W_q . vec(Y^C_i) -> round to bf16
+//   Y^C_i (LCB, Eq. 6) -> [round to bf16 if round_y] -> Q_i = W_q . vec(Y^C_i) -> round to bf16
 //   -> DCA over request m_i's keys with H heads of size dh.
+// round_y = 1: Y^C is stored in bf16 between the LCB and the projection (the unfused chain);
+// round_y = 0: the projection consumes the exact LCB output (a chain that never stores Y^C).
 // Outputs: y_cand [n_sel, o_c, d] (before rounding), q_out [n_sel, H*dh] (before rounding),
 // o [n_sel, H, dh], lse [n_sel, H].
-int rocs_oracle_chain(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n_c, int64_t d, int64_t o_r,
+static int chain_impl(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n_c, int64_t d, int64_t o_r,
                       int64_t o_c, const uint16_t* x_req, const uint16_t* x_cand, const uint16_t* w_rr,
                       const uint16_t* w_cr, const uint16_t* w_cc, const uint16_t* w_q, const int32_t* seq_off,
                       int64_t H, int64_t dh, double scale, const uint16_t* K, const uint16_t* V, int64_t n_sel,
-                      const int64_t* sel_cand, double* y_cand, double* q_out, double* o, double* lse, int nthreads) {
+                      const int64_t* sel_cand, double* y_cand, double* q_out, double* o, double* lse, int round_y,
+                      int nthreads) {
   if (!csr_ok(cand_off, R, -1) || !csr_ok(seq_off, R, -1)) return ORC_BAD_OFFSETS;
   set_threads(nthreads);
   const LcbDims D{n_r, n_c, d, o_r, o_c};
@@ -373,7 +376,7 @@ int rocs_oracle_chain(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n
     double* yc = y_cand + k * n_in;
     if (!lcb_candidate(D, 1, x_req, x_cand, W, i, r, yc)) bad |= 1;
     std::vector<double> yb((size_t)n_in), qb((size_t)n_out);
-    for (int64_t j = 0; j < n_in; ++j) yb[(size_t)j] = round_bf16(yc[j]);
+    for (int64_t j = 0; j < n_in; ++j) yb[(size_t)j] = round_y ? round_bf16(yc[j]) : yc[j];
     for (int64_t n = 0; n < n_out; ++n) {
       double acc = 0.0;
       for (int64_t j = 0; j < n_in; ++j) acc += widen(w_q, 1, n * n_in + j) * yb[(size_t)j];
@@ -383,6 +386,43 @@ int rocs_oracle_chain(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n
     dca_candidate(DD, nullptr, K, V, i, seq_off[r], seq_off[r + 1], qb.data(), o + k * n_out, lse + k * H);
   }
   return bad ? ORC_ISOLATION : ORC_OK;
+}
+
+int rocs_oracle_chain(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n_c, int64_t d, int64_t o_r,
+                      int64_t o_c, const uint16_t* x_req, const uint16_t* x_cand, const uint16_t* w_rr,
+                      const uint16_t* w_cr, const uint16_t* w_cc, const uint16_t* w_q, const int32_t* seq_off,
+                      int64_t H, int64_t dh, double scale, const uint16_t* K, const uint16_t* V, int64_t n_sel,
+                      const int64_t* sel_cand, double* y_cand, double* q_out, double* o, double* lse, int nthreads) {
+  return chain_impl(R, cand_off, n_r, n_c, d, o_r, o_c, x_req, x_cand, w_rr, w_cr, w_cc, w_q, seq_off, H, dh, scale,
+                    K, V, n_sel, sel_cand, y_cand, q_out, o, lse, 1, nthreads);
+}
+
+int rocs_oracle_chain_exact(int64_t R, const int32_t* cand_off, int64_t n_r, int64_t n_c, int64_t d, int64_t o_r,
+                            int64_t o_c, const uint16_t* x_req, const uint16_t* x_cand, const uint16_t* w_rr,
+                            const uint16_t* w_cr, const uint16_t* w_cc, const uint16_t* w_q, const int32_t* seq_off,
+                            int64_t H, int64_t dh, double scale, const uint16_t* K, const uint16_t* V, int64_t n_sel,
+                            const int64_t* sel_cand, double* y_cand, double* q_out, double* o, double* lse,
+                            int nthreads) {
+  return chain_impl(R, cand_off, n_r, n_c, d, o_r, o_c, x_req, x_cand, w_rr, w_cr, w_cc, w_q, seq_off, H, dh, scale,
+                    K, V, n_sel, sel_cand, y_cand, q_out, o, lse, 0, nthreads);
+}
+
+// The projection weight folded with W_CC (the linear maps compose):
+//   W_q vec(W_CC X) = W_fold vec(X),   W_fold[k, n*d + c] = sum_o W_q[k, o*d + c] W_CC[o, n]
+// w_q [n_out, o_c*d] bf16, w_cc [o_c, n_c] bf16 -> w_fold [n_out, n_c*d] in fp64.
+int rocs_oracle_chain_fold(int64_t n_out, int64_t o_c, int64_t n_c, int64_t d, const uint16_t* w_q,
+                           const uint16_t* w_cc, double* w_fold, int nthreads) {
+  if (n_out < 0 || o_c < 0 || n_c < 0 || d < 0) return ORC_INVALID;
+  set_threads(nthreads);
+#pragma omp parallel for schedule(static)
+  for (int64_t k = 0; k < n_out; ++k)
+    for (int64_t n = 0; n < n_c; ++n)
+      for (int64_t c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int64_t o = 0; o < o_c; ++o) acc += widen(w_q, 1, k * o_c * d + o * d + c) * widen(w_cc, 1, o * n_c + n);
+        w_fold[(k * n_c + n) * d + c] = acc;
+      }
+  return ORC_OK;
 }
 
 // DCA block (section 3.2, Eq. (13)), both query groups, for the selected requests / candidates.

@@ -616,3 +616,60 @@ def test_pad_transform_leaves_the_computation_unchanged(oracle_mod):
     assert np.array_equal(oracle_mod.unpad_cols(yp, 30), y)
     wp = oracle_mod.pad_cols(w.reshape(11, 3, 30), 32).reshape(11, 96)
     assert np.array_equal(yp.reshape(7, 96) @ wp.T, y.reshape(7, 90) @ w.T)
+
+
+# ------------------------------------------------------------------------------ split chain (f2)
+# The chain that never stores Y^C: Q_i = W_q vec(Y^C_i) with the exact LCB output, which the IKBO
+# decomposition splits into W_q vec(Z_{m_i}) (once per request) + W_fold vec(X^C_i).
+def _bf16_bits(a):
+    return (np.asarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_chain_exact_equals_rounded_chain_when_y_is_exact(oracle_mod):
+    # small integers everywhere: every Y^C entry is an exact bf16 value, so rounding it changes nothing
+    ci = _shrink_chain(_small_chain(44))
+    x = ci.lcb
+    rs = np.random.RandomState(3)
+    for name in ("x_req", "x_cand"):
+        setattr(x, name, _bf16_bits(rs.randint(-2, 3, size=getattr(x, name).shape)))
+    for name in ("w_rr", "w_cr", "w_cc"):
+        setattr(x, name, _bf16_bits(rs.randint(-1, 2, size=getattr(x, name).shape)))
+    sel = np.arange(x.C)
+    a = oracle_mod.chain(ci, sel, round_y=True)
+    b = oracle_mod.chain(ci, sel, round_y=False)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+
+
+def test_chain_exact_query_matches_library(oracle_mod):
+    ci = _shrink_chain(_small_chain(45))
+    x = ci.lcb
+    y, qo, _, _ = oracle_mod.chain(ci, np.arange(x.C), round_y=False)
+    w = lambda a: ri.bf16_to_f32(a).astype(np.float64)
+    m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+    yc = np.einsum("on,ind->iod", w(x.w_cr), w(x.x_req)[m]) + np.einsum("on,ind->iod", w(x.w_cc), w(x.x_cand))
+    assert np.max(np.abs(y - yc)) <= 1e-12 * np.max(np.abs(yc))
+    q = yc.reshape(x.C, -1) @ w(ci.w_q).T
+    assert np.max(np.abs(qo - q)) <= 1e-12 * np.max(np.abs(q))
+
+
+def test_split_projection_identity(oracle_mod):
+    # Q_i = W_q vec(Z_{m_i}) + W_fold vec(X^C_i): pins the fold's index map (a transposed fold fails)
+    ci = _shrink_chain(_small_chain(46))
+    x = ci.lcb
+    _, qo, _, _ = oracle_mod.chain(ci, np.arange(x.C), round_y=False)
+    w = lambda a: ri.bf16_to_f32(a).astype(np.float64)
+    wf = oracle_mod.chain_fold(ci.w_q, x.w_cc, x.d)
+    assert wf.shape == (ci.H * ci.dh, x.n_c * x.d)
+    m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
+    z = np.einsum("on,rnd->rod", w(x.w_cr), w(x.x_req)).reshape(x.R, -1)
+    q = (z @ w(ci.w_q).T)[m] + w(x.x_cand).reshape(x.C, -1) @ wf.T
+    assert np.max(np.abs(qo - q)) <= 1e-12 * np.max(np.abs(q))
+
+
+def test_chain_fold_closed_form(oracle_mod):
+    # W_CC = identity: the folded weight is W_q itself
+    n_out, o_c, d = 6, 4, 3
+    wq = ri.normal(9, 1, (n_out, o_c * d))
+    eye = _bf16_bits(np.eye(o_c))
+    assert np.array_equal(oracle_mod.chain_fold(wq, eye, d), ri.bf16_to_f32(wq).astype(np.float64))
