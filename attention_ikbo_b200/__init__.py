@@ -19,17 +19,23 @@ Operations ("ROCS: Request-Oriented Compute Sharing ...", arXiv:2607.27744):
   * :func:`rocs_dca_block_forward` -- both query groups of Eq. (13) with the K/V projections
     done once per request (section 4.1).
   * :func:`rocs_proj_forward` -- linear query projection of the chained block (Eq. 12).
+  * :func:`rocs_chain_split_forward` / :func:`chain_split_forward` -- the chain with the projection
+    split over the IKBO decomposition (request term once per request, W_q folded with W_CC by
+    :func:`rocs_chain_prepare_weights`), so Y^C is never written.
 """
 from ._binding import (  # noqa: F401
     ROCS_BF16,
     ROCS_F32,
     RocsError,
     chain_forward,
+    chain_split_forward,
     last_launch_count,
     lib_path,
     load_library,
     offsets,
     rocs_align_cols,
+    rocs_chain_prepare_weights,
+    rocs_chain_split_forward,
     rocs_dca_block_forward,
     rocs_dca_forward,
     rocs_dca_forward_expand,

@@ -45,6 +45,18 @@ class FmArgs(ctypes.Structure):
                 ("ld_req", _i64), ("ld_cand", _i64), ("workspace", _vp), ("workspace_bytes", _sz)]
 
 
+class ChainWeightsArgs(ctypes.Structure):
+    _fields_ = [("n_out", _i64), ("o_r", _i64), ("o_c", _i64), ("n_r", _i64), ("n_c", _i64), ("d", _i64),
+                ("w_q", _vp), ("w_rr", _vp), ("w_cr", _vp), ("w_cc", _vp), ("w_fold", _vp), ("w_rs", _vp)]
+
+
+class ChainSplitArgs(ctypes.Structure):
+    _fields_ = [("R", _i64), ("n_r", _i64), ("n_c", _i64), ("d", _i64), ("o_r", _i64), ("o_c", _i64),
+                ("n_out", _i64), ("cand_off_dev", _vp), ("cand_off_host", _vp), ("x_req", _vp), ("x_cand", _vp),
+                ("w_rs", _vp), ("w_q", _vp), ("w_fold", _vp), ("y_req", _vp), ("q", _vp), ("workspace", _vp),
+                ("workspace_bytes", _sz)]
+
+
 class DcaArgs(ctypes.Structure):
     _fields_ = [("R", _i64), ("q", _i64), ("H", _i64), ("dh", _i64), ("scale", _f32),
                 ("cand_off_dev", _vp), ("cand_off_host", _vp), ("seq_off_dev", _vp), ("seq_off_host", _vp),
@@ -84,7 +96,8 @@ def load_library():
                            ("rocs_dca_workspace_size", [P(DcaArgs)]), ("rocs_proj_workspace_size", [P(ProjArgs)]),
                            ("rocs_dca_expand_workspace_size", [P(DcaArgs), _i64]),
                            ("rocs_dca_block_workspace_size", [P(DcaBlockArgs)]),
-                           ("rocs_fm_workspace_size", [P(FmArgs)])]:
+                           ("rocs_fm_workspace_size", [P(FmArgs)]),
+                           ("rocs_chain_split_workspace_size", [P(ChainSplitArgs)])]:
             getattr(lib, name).restype = _sz
             getattr(lib, name).argtypes = argt
         for name, argt in [("rocs_lcb_forward", [P(LcbArgs), _vp]), ("rocs_lcb_forward_expand", [P(LcbArgs), _vp]),
@@ -95,6 +108,8 @@ def load_library():
                            ("rocs_dca_forward_expand", [P(DcaArgs), _i64, _vp]),
                            ("rocs_dca_block_forward", [P(DcaBlockArgs), _vp]),
                            ("rocs_fm_forward", [P(FmArgs), _vp]),
+                           ("rocs_chain_prepare_weights", [P(ChainWeightsArgs), _vp]),
+                           ("rocs_chain_split_forward", [P(ChainSplitArgs), _vp]),
                            ("rocs_pad_cols", [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _vp]),
                            ("rocs_read_status", [_vp, _vp, P(_i32), P(_i32)])]:
             getattr(lib, name).restype = ctypes.c_int
@@ -454,3 +469,66 @@ def rocs_fm_forward(x_req, x_cand, cand_off, y_req=None, y_cand=None, ld_req=0, 
     _check(lib.rocs_fm_forward(ctypes.byref(a), _stream(stream)), "rocs_fm_forward")
     rocs_fm_forward.last_workspace = ws
     return y_req, y_cand
+
+
+def rocs_chain_prepare_weights(w_q, w_rr, w_cr, w_cc, d, stream=None):
+    """Once per model: ``(w_fold [n_out, n_c*d], w_rs [o_r + o_c, n_r])`` for :func:`rocs_chain_split_forward`."""
+    lib = load_library()
+    for t in (w_q, w_rr, w_cr, w_cc):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16):
+            raise RocsError(1, "chain weights must be contiguous CUDA bf16 tensors")
+    n_out, (o_r, n_r), (o_c, n_c) = w_q.shape[0], w_rr.shape, w_cc.shape
+    w_fold = torch.empty((n_out, n_c * d), dtype=torch.bfloat16, device=w_q.device)
+    w_rs = torch.empty((o_r + o_c, n_r), dtype=torch.bfloat16, device=w_q.device)
+    a = ChainWeightsArgs(n_out=n_out, o_r=o_r, o_c=o_c, n_r=n_r, n_c=n_c, d=d, w_q=w_q.data_ptr(),
+                         w_rr=w_rr.data_ptr(), w_cr=w_cr.data_ptr(), w_cc=w_cc.data_ptr(), w_fold=w_fold.data_ptr(),
+                         w_rs=w_rs.data_ptr())
+    _check(lib.rocs_chain_prepare_weights(ctypes.byref(a), _stream(stream)), "rocs_chain_prepare_weights")
+    return w_fold, w_rs
+
+
+def rocs_chain_split_forward(x_req, x_cand, w_rs, w_q, w_fold, cand_off, o_r, y_req=None, q=None, workspace=None,
+                             stream=None):
+    """Split chain queries: ``(y_req [R, o_r + o_c, d] = [Y^R; Z], q [C, n_out])``; see the header."""
+    lib = load_library()
+    dev = x_req.device
+    off_d, off_h = _offsets(cand_off, dev)
+    R, n_r, d = x_req.shape
+    C = int(off_h[-1])
+    n_c = x_cand.shape[1]
+    o_c = w_rs.shape[0] - o_r
+    n_out = w_q.shape[0]
+    if y_req is None:
+        y_req = torch.empty((R, o_r + o_c, d), dtype=torch.bfloat16, device=dev)
+    if q is None:
+        q = torch.empty((C, n_out), dtype=torch.bfloat16, device=dev)
+    for t in (x_req, x_cand, w_rs, w_q, w_fold, y_req, q):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16):
+            raise RocsError(1, "split chain tensors must be contiguous CUDA bf16 tensors")
+    a = ChainSplitArgs(R=R, n_r=n_r, n_c=n_c, d=d, o_r=o_r, o_c=o_c, n_out=n_out, cand_off_dev=off_d.data_ptr(),
+                       cand_off_host=off_h.ctypes.data, x_req=x_req.data_ptr(),
+                       x_cand=x_cand.data_ptr() if C else None, w_rs=w_rs.data_ptr(), w_q=w_q.data_ptr(),
+                       w_fold=w_fold.data_ptr(), y_req=y_req.data_ptr(), q=q.data_ptr() if C else None)
+    nbytes = lib.rocs_chain_split_workspace_size(ctypes.byref(a))
+    if nbytes == 0:
+        _check(lib.rocs_chain_split_forward(ctypes.byref(a), _stream(stream)), "rocs_chain_split_forward")
+    ws = _workspace(nbytes, dev, workspace)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check(lib.rocs_chain_split_forward(ctypes.byref(a), _stream(stream)), "rocs_chain_split_forward")
+    rocs_chain_split_forward.last_workspace = ws
+    return y_req, q
+
+
+def chain_split_forward(x_req, x_cand, w_rs, w_q, w_fold, cand_off, o_r, k_t, v_t, seq_off, heads, head_dim, scale,
+                        stream=None, workspaces=None):
+    """Split chained block: queries from :func:`rocs_chain_split_forward` (Y^C never written), then IKBO-DCA.
+
+    Returns ``(y_req, q, o, lse)``.
+    """
+    ws = workspaces or {}
+    y_req, q = rocs_chain_split_forward(x_req, x_cand, w_rs, w_q, w_fold, cand_off, o_r, workspace=ws.get("split"),
+                                        stream=stream)
+    C = q.shape[0]
+    o, lse = rocs_dca_forward(q.view(C, heads, head_dim), k_t, v_t, cand_off, seq_off, 1, scale,
+                              workspace=ws.get("dca"), stream=stream)
+    return y_req, q, o, lse

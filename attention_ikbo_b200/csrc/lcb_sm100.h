@@ -66,13 +66,19 @@ cudaError_t launch_dca_schedule(const DcaSchedParams& p, cudaStream_t st);
 
 // Dense projection GEMM  out[M, N] = in[M, K] . W[N, K]^T  (bf16 in/out, fp32 accumulate).
 struct ProjParams {
-  CUtensorMap tm_a;    // in  [M, K], box {64, 128}
+  CUtensorMap tm_a;    // in  [M, K] (row stride lda), box {64, 128}
   CUtensorMap tm_b;    // W   [N, K], box {64, 256}
-  __nv_bfloat16* out;  // [M, N]
+  __nv_bfloat16* out;  // [M, N] bf16, or null when out_f32 is given
+  float* out_f32;      // [M, N] fp32 output instead of bf16 (or null)
+  const float* add;    // IKBO broadcast-add: out[i, :] += add[m_i, :] with m_i from add_off (or null)
+  const int32_t* add_off;  // [add_R + 1] CSR: rows add_off[r] .. add_off[r+1]-1 belong to r
   WsHeader* ws;
-  int M, N, K;
+  int M, N, K, add_R;
   long long wait_limit_ns;
 };
+// W_fold[k, n*d + c] = sum_o W_q[k, o*d + c] W_CC[o, n]  (fp32 accumulate, bf16 out)
+cudaError_t launch_chain_fold(const __nv_bfloat16* w_q, const __nv_bfloat16* w_cc, __nv_bfloat16* w_fold, int n_out,
+                              int o_c, int n_c, int d, cudaStream_t st);
 cudaError_t launch_proj_sm100(const ProjParams& p, int grid, cudaStream_t st);
 
 // IKBO masked factorization machine (bf16 in, fp32 accumulate, bf16 out in aligned rows).

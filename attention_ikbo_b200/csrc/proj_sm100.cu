@@ -7,7 +7,9 @@
 // Persistent CTAs take output tiles of 128 x 256 in (m, n) order with n innermost so the
 // CTAs that run together share one 128-row block of `in` through L2.  Warp 0 issues TMA
 // loads (K-blocks of 64, 4-stage ring), warp 1 issues tcgen05.mma (M=128, N=256, K=16),
-// warps 2-5 drain the double-buffered TMEM accumulator and store bf16 rows.
+// warps 2-5 drain the double-buffered TMEM accumulator and store bf16 (or fp32) rows, optionally
+// adding a per-request row of an fp32 matrix first (the IKBO broadcast-add of the split chain:
+// row i gets add[m_i, :], m_i from CSR offsets).
 #include "lcb_sm100.h"
 
 namespace rocs {
@@ -117,25 +119,52 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_proj_sm100_kernel(const __gr
     const int quarter = warp & 3;
     const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
     uint32_t ab = 0, aph = 0;
+    int m_row = -1, m_row_for = -1;  // request of this thread's row (IKBO broadcast-add)
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int m0 = (t / nt) * BM, n0 = (t % nt) * BN;
       if (!mbar_wait(&acc_full[ab], aph, ctl, 904)) break;
       tc_fence_after();
       const int row = m0 + 32 * quarter + (int)lane;
-      __nv_bfloat16* orow = p.out + (size_t)row * p.N + n0;
+      if (p.add && row < p.M && row != m_row_for) {  // last r with add_off[r] <= row
+        int lo = 0, hi = p.add_R - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (__ldg(p.add_off + mid) <= row) lo = mid; else hi = mid - 1;
+        }
+        m_row = lo;
+        m_row_for = row;
+      }
+      const float* arow = p.add ? p.add + (size_t)m_row * p.N + n0 : nullptr;
 #pragma unroll 1
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t v[32];
         tmem_ld32(tmem_base + t_lane + ab * BN + cc * 32, v);
         tmem_ld_wait();
         if (row < p.M) {
+          if (arow) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            st_global_v4(orow + cc * 32 + 8 * k,
-                         pack_bf16x2(__uint_as_float(v[8 * k + 0]), __uint_as_float(v[8 * k + 1])),
-                         pack_bf16x2(__uint_as_float(v[8 * k + 2]), __uint_as_float(v[8 * k + 3])),
-                         pack_bf16x2(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5])),
-                         pack_bf16x2(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7])));
+            for (int k = 0; k < 8; ++k) {
+              const float4 a4 = __ldg(reinterpret_cast<const float4*>(arow + cc * 32) + k);
+              v[4 * k + 0] = __float_as_uint(__uint_as_float(v[4 * k + 0]) + a4.x);
+              v[4 * k + 1] = __float_as_uint(__uint_as_float(v[4 * k + 1]) + a4.y);
+              v[4 * k + 2] = __float_as_uint(__uint_as_float(v[4 * k + 2]) + a4.z);
+              v[4 * k + 3] = __float_as_uint(__uint_as_float(v[4 * k + 3]) + a4.w);
+            }
+          }
+          if (p.out_f32) {
+            float* frow = p.out_f32 + (size_t)row * p.N + n0 + cc * 32;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) st_global_v4(frow + 4 * k, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          } else {
+            __nv_bfloat16* orow = p.out + (size_t)row * p.N + n0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              st_global_v4(orow + cc * 32 + 8 * k,
+                           pack_bf16x2(__uint_as_float(v[8 * k + 0]), __uint_as_float(v[8 * k + 1])),
+                           pack_bf16x2(__uint_as_float(v[8 * k + 2]), __uint_as_float(v[8 * k + 3])),
+                           pack_bf16x2(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5])),
+                           pack_bf16x2(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7])));
+          }
         }
       }
       tc_fence_before();
@@ -151,6 +180,25 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_proj_sm100_kernel(const __gr
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+}
+
+// one CTA per (k, n), one thread per c: sum over o of W_q[k, o*d + c] W_CC[o, n]
+__global__ void rocs_chain_fold_kernel(const __nv_bfloat16* __restrict__ w_q, const __nv_bfloat16* __restrict__ w_cc,
+                                       __nv_bfloat16* __restrict__ w_fold, int o_c, int n_c, int d) {
+  const int kn = blockIdx.x, k = kn / n_c, n = kn - k * n_c;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float acc = 0.0f;
+    for (int o = 0; o < o_c; ++o)
+      acc = fmaf(__bfloat162float(w_q[((size_t)k * o_c + o) * d + c]), __bfloat162float(w_cc[(size_t)o * n_c + n]), acc);
+    w_fold[((size_t)k * n_c + n) * d + c] = __float2bfloat16_rn(acc);
+  }
+}
+
+cudaError_t launch_chain_fold(const __nv_bfloat16* w_q, const __nv_bfloat16* w_cc, __nv_bfloat16* w_fold, int n_out,
+                              int o_c, int n_c, int d, cudaStream_t st) {
+  const int threads = d < 1024 ? ((d + 31) / 32) * 32 : 1024;
+  rocs_chain_fold_kernel<<<n_out * n_c, threads, 0, st>>>(w_q, w_cc, w_fold, o_c, n_c, d);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_proj_sm100(const ProjParams& p, int grid, cudaStream_t st) {

@@ -655,6 +655,30 @@ size_t rocs_proj_workspace_size(const rocs_proj_args* a) {
   return sizeof(WsHeader);
 }
 
+// out[M, N] = in[M, K] (row stride lda) . w[N, K]^T (+ add[m_i, :]), bf16 or fp32 out; M > 0
+static int proj_run(const void* in, int64_t lda, const void* w, void* out_bf16, float* out_f32, const float* add,
+                    const int32_t* add_off, int64_t add_R, int64_t M, int64_t N, int64_t K, WsHeader* hdr,
+                    cudaStream_t st) {
+  ProjParams p;
+  std::memset(&p, 0, sizeof(p));
+  bool ok = tmap_bf16(&p.tm_a, in, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2, 64, 128);
+  ok &= tmap_bf16(&p.tm_b, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, 64, 256);
+  if (!ok) return ROCS_ERR_CUDA;
+  p.out = static_cast<__nv_bfloat16*>(out_bf16);
+  p.out_f32 = out_f32;
+  p.add = add;
+  p.add_off = add_off;
+  p.add_R = (int)add_R;
+  p.ws = hdr;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.wait_limit_ns = kDefaultWaitLimitNs;
+  const int64_t tiles = ((M + 127) / 128) * (N / 256);
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  return launch_proj_sm100(p, grid, st) == cudaSuccess ? ROCS_OK : ROCS_ERR_CUDA;
+}
+
 int rocs_proj_forward(const rocs_proj_args* a, rocs_stream_t stream) {
   if (!a || a->M < 0 || a->N <= 0 || a->K <= 0) return ROCS_ERR_INVALID_ARG;
   if (a->N % 256 || a->K % 64) return ROCS_ERR_UNSUPPORTED;
@@ -670,21 +694,101 @@ int rocs_proj_forward(const rocs_proj_args* a, rocs_stream_t stream) {
     g_last_launches = 0;
     return ROCS_OK;
   }
-  ProjParams p;
-  std::memset(&p, 0, sizeof(p));
-  bool ok = tmap_bf16(&p.tm_a, a->in, a->K, a->M, a->K * 2, 64, 128);
-  ok &= tmap_bf16(&p.tm_b, a->w, a->K, a->N, a->K * 2, 64, 256);
-  if (!ok) return ROCS_ERR_CUDA;
-  p.out = static_cast<__nv_bfloat16*>(a->out);
-  p.ws = static_cast<WsHeader*>(a->workspace);
-  p.M = (int)a->M;
-  p.N = (int)a->N;
-  p.K = (int)a->K;
-  p.wait_limit_ns = kDefaultWaitLimitNs;
-  const int64_t tiles = ((a->M + 127) / 128) * (a->N / 256);
-  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  if (launch_proj_sm100(p, grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  const int rc = proj_run(a->in, a->K, a->w, a->out, nullptr, nullptr, nullptr, 0, a->M, a->N, a->K,
+                          static_cast<WsHeader*>(a->workspace), st);
+  if (rc == ROCS_OK) g_last_launches = 1;
+  return rc;
+}
+
+// ---------------------------------------------------------------- split chain
+int rocs_chain_prepare_weights(const rocs_chain_weights_args* a, rocs_stream_t stream) {
+  if (!a || a->n_out <= 0 || a->o_r <= 0 || a->o_c <= 0 || a->n_r <= 0 || a->n_c <= 0 || a->d <= 0)
+    return ROCS_ERR_INVALID_ARG;
+  if (a->n_out * a->n_c >= (int64_t(1) << 31) || a->d > 4096 || a->o_c > 4096) return ROCS_ERR_UNSUPPORTED;
+  const void* ptrs[] = {a->w_q, a->w_rr, a->w_cr, a->w_cc, a->w_fold, a->w_rs};
+  for (const void* p : ptrs)
+    if (!p || !al16(p)) return ROCS_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t rr = (size_t)a->o_r * a->n_r * 2, cr = (size_t)a->o_c * a->n_r * 2;
+  if (cudaMemcpyAsync(a->w_rs, a->w_rr, rr, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(static_cast<uint8_t*>(a->w_rs) + rr, a->w_cr, cr, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return ROCS_ERR_CUDA;
+  if (launch_chain_fold(static_cast<const __nv_bfloat16*>(a->w_q), static_cast<const __nv_bfloat16*>(a->w_cc),
+                        static_cast<__nv_bfloat16*>(a->w_fold), (int)a->n_out, (int)a->o_c, (int)a->n_c, (int)a->d,
+                        st) != cudaSuccess)
+    return ROCS_ERR_CUDA;
   g_last_launches = 1;
+  return ROCS_OK;
+}
+
+static int split_validate(const rocs_chain_split_args* a, int64_t* C) {
+  if (!a) return ROCS_ERR_INVALID_ARG;
+  if (a->R < 0 || a->n_out <= 0) return ROCS_ERR_INVALID_ARG;
+  if (a->n_out % 256 || (a->o_c * a->d) % 64 || (a->n_c * a->d) % 64) return ROCS_ERR_UNSUPPORTED;
+  // the request GEMM runs as an LCB with no candidates over the stacked [W_RR; W_CR]
+  rocs_lcb_args l;
+  std::memset(&l, 0, sizeof(l));
+  l.R = a->R; l.n_r = a->n_r; l.n_c = a->n_c; l.d = a->d; l.o_r = a->o_r + a->o_c; l.o_c = a->o_c;
+  l.dtype = ROCS_BF16; l.cand_off_dev = a->cand_off_dev; l.cand_off_host = a->cand_off_host;
+  l.x_req = a->x_req; l.x_cand = a->x_cand; l.w_rr = a->w_rs; l.w_cr = a->w_rs; l.w_cc = a->w_rs;
+  l.y_req = a->y_req; l.y_cand = a->q;
+  int rc = lcb_validate(&l, C);
+  if (rc) return rc;
+  if (*C * a->n_c >= (int64_t(1) << 31) || *C * a->n_out >= (int64_t(1) << 31)) return ROCS_ERR_UNSUPPORTED;
+  if (a->R > 0 && (!a->w_q || !al16(a->w_q))) return ROCS_ERR_INVALID_ARG;
+  if (*C > 0 && (!a->w_fold || !a->q || !al16(a->w_fold) || !al16(a->q))) return ROCS_ERR_INVALID_ARG;
+  return ROCS_OK;
+}
+
+static size_t split_bytes(const rocs_chain_split_args* a) {
+  // [LCB workspace: header, flags, Z fp32 (request GEMM, discarded)] [q^R fp32 [R, n_out]]
+  return a256(sizeof(WsHeader) + lcb_body(a->R, a->o_c, a->d).body) + (size_t)a->R * a->n_out * sizeof(float);
+}
+
+size_t rocs_chain_split_workspace_size(const rocs_chain_split_args* a) {
+  int64_t C;
+  if (split_validate(a, &C) != ROCS_OK) return 0;
+  return split_bytes(a);
+}
+
+int rocs_chain_split_forward(const rocs_chain_split_args* a, rocs_stream_t stream) {
+  int64_t C = 0;
+  int rc = split_validate(a, &C);
+  if (rc) return rc;
+  if (!a->workspace || a->workspace_bytes < split_bytes(a) || (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ROCS_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
+  float* q_req = reinterpret_cast<float*>(static_cast<uint8_t*>(a->workspace) +
+                                          a256(sizeof(WsHeader) + lcb_body(a->R, a->o_c, a->d).body));
+  rocs_lcb_args l;
+  std::memset(&l, 0, sizeof(l));
+  l.R = a->R; l.n_r = a->n_r; l.n_c = a->n_c; l.d = a->d; l.o_r = a->o_r + a->o_c; l.o_c = a->o_c;
+  l.dtype = ROCS_BF16; l.cand_off_dev = a->cand_off_dev; l.cand_off_host = a->cand_off_host;
+  l.x_req = a->x_req; l.w_rr = a->w_rs; l.w_cr = static_cast<const uint8_t*>(a->w_rs) + (size_t)a->o_r * a->n_r * 2;
+  l.w_cc = a->w_rs; l.y_req = a->y_req;
+  int launches = 0;
+  // 1. [Y^R_r; Z_r] = [W_RR; W_CR] X^R_r once per request (an LCB call without candidates)
+  rc = lcb_run(&l, 0, hdr, reinterpret_cast<uint8_t*>(hdr + 1), st, &launches);
+  if (rc) return rc;
+  if (a->R == 0) {
+    g_last_launches = launches;
+    return ROCS_OK;
+  }
+  // 2. q^R_r = W_q vec(Z_r) in fp32 (Z_r = rows o_r.. of the request block, row stride (o_r + o_c) d)
+  const int64_t zd = a->o_c * a->d, ld = (a->o_r + a->o_c) * a->d;
+  rc = proj_run(static_cast<const uint8_t*>(a->y_req) + (size_t)a->o_r * a->d * 2, ld, a->w_q, nullptr, q_req, nullptr,
+                nullptr, 0, a->R, a->n_out, zd, hdr, st);
+  if (rc) return rc;
+  ++launches;
+  // 3. Q_i = W_fold vec(X^C_i) + q^R_{m_i}: the candidate GEMM with the broadcast-add fused
+  if (C > 0) {
+    rc = proj_run(a->x_cand, a->n_c * a->d, a->w_fold, a->q, nullptr, q_req, a->cand_off_dev, a->R, C, a->n_out,
+                  a->n_c * a->d, hdr, st);
+    if (rc) return rc;
+    ++launches;
+  }
+  g_last_launches = launches;
   return ROCS_OK;
 }
 

@@ -426,6 +426,61 @@ class ProjPart(Part):
         return time.perf_counter() - t0, len(sel) / self.M
 
 
+class SplitPart(Part):
+    """Split chain queries: [Y^R; Z] = [W_RR; W_CR] X^R per request, q^R = W_q vec(Z), then
+    Q = W_fold vec(X^C) + q^R[m] (three launches; Y^C never written).  The folded weights are model
+    preprocessing, prepared once before timing."""
+    bound, kernel = "tensor", "proj"
+
+    def __init__(self, ci: ri.ChainInputs):
+        self.ci, self.name = ci, "chain_split"
+        x = ci.lcb
+        self.units = x.C
+        self.N = ci.H * ci.dh
+
+    def flops(self):
+        x = self.ci.lcb
+        return (acc.proj_flops(x.R * (x.o_r + x.o_c), x.d, x.n_r) + acc.proj_flops(x.R, self.N, x.o_c * x.d)
+                + acc.proj_flops(x.C, self.N, x.n_c * x.d))
+
+    def bytes(self):
+        x = self.ci.lcb
+        return 2 * (x.R * x.n_r * x.d + x.C * x.n_c * x.d + (x.o_r + x.o_c) * x.n_r + self.N * x.o_c * x.d
+                    + self.N * x.n_c * x.d + x.R * (x.o_r + x.o_c) * x.d + x.C * self.N)
+
+    def to_device(self, ikbo, torch, dev):
+        ci, x = self.ci, self.ci.lcb
+        self.h_in = [_pin(torch, a) for a in (x.x_req, x.x_cand)]
+        self.d_in = [h.to(dev) for h in self.h_in]
+        self.w_q = _to_dev(torch, ci.w_q, dev)
+        self.w_fold, self.w_rs = ikbo.rocs_chain_prepare_weights(
+            self.w_q, *[_to_dev(torch, a, dev) for a in (x.w_rr, x.w_cr, x.w_cc)], x.d)
+        self.off = ikbo.offsets(x.cand_off, dev)
+        self.h_off = _pin(torch, x.cand_off)
+        self.y_req, self.out = ikbo.rocs_chain_split_forward(*self.d_in, self.w_rs, self.w_q, self.w_fold, self.off,
+                                                             x.o_r)
+        self.ws = ikbo.rocs_chain_split_forward.last_workspace
+        self.h_out = [torch.empty(self.y_req.shape, dtype=self.y_req.dtype, pin_memory=True)]
+
+    def run(self, ikbo):
+        ikbo.rocs_chain_split_forward(*self.d_in, self.w_rs, self.w_q, self.w_fold, self.off, self.ci.lcb.o_r,
+                                      self.y_req, self.out, workspace=self.ws)
+        return ikbo.last_launch_count()
+
+    def h2d(self):
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+        self.off[0].copy_(self.h_off, non_blocking=True)
+        return sum(h.numel() * h.element_size() for h in self.h_in) + self.h_off.numel() * 4
+
+    def d2h(self):
+        self.h_out[0].copy_(self.y_req, non_blocking=True)
+        return self.h_out[0].numel() * self.h_out[0].element_size()
+
+    def status(self, ikbo):
+        return ikbo.rocs_read_status(self.ws)
+
+
 def _pin(torch, a):
     t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16 else np.ascontiguousarray(a))
     if a.dtype == np.uint16:
@@ -442,8 +497,8 @@ class ChainOracle:
 
     name = "chain"
 
-    def __init__(self, ci):
-        self.ci = ci
+    def __init__(self, ci, round_y=True):
+        self.ci, self.round_y = ci, round_y
 
     def oracle_sample(self, oracle, n, seed):
         ci = self.ci
@@ -457,7 +512,7 @@ class ChainOracle:
         w_dca = 4 * ci.H * ci.dh * L[m]
         frac = float((w_fixed + w_dca[sel]).sum()) / float((w_fixed + w_dca).sum())
         t0 = time.perf_counter()
-        oracle.chain(ci, sel)
+        oracle.chain(ci, sel, round_y=self.round_y)
         return time.perf_counter() - t0, frac
 
 
@@ -465,7 +520,9 @@ _CHAIN = {}
 
 
 def oracle_parts(workload, parts):
-    return [ChainOracle(_CHAIN["ci"])] if workload == "chain" else parts
+    if workload in ("chain", "chain_split"):
+        return [ChainOracle(_CHAIN["ci"], round_y=workload == "chain")]
+    return parts
 
 
 def make_parts(workload):
@@ -491,13 +548,23 @@ def make_parts(workload):
         dca_in = ri.DcaInputs("chain_dca", x.cand_off, ci.seq_off, 1, ci.H, ci.dh, ci.scale, qdummy, ci.k_t, ci.v_t)
         _CHAIN["ci"] = ci
         return [lcb, ProjPart(ci, lcb), DcaPart(dca_in, "chain_dca")]
+    if workload == "chain_split":
+        ci = ri.chain()
+        x = ci.lcb
+        qdummy = np.zeros((0,), np.uint16)
+        dca_in = ri.DcaInputs("chain_dca", x.cand_off, ci.seq_off, 1, ci.H, ci.dh, ci.scale, qdummy, ci.k_t, ci.v_t)
+        _CHAIN["ci"] = ci
+        return [SplitPart(ci), DcaPart(dca_in, "chain_dca")]
     raise ValueError(workload)
 
 
 def workload_config(workload, parts):
-    if workload == "chain":
+    if workload in ("chain", "chain_split"):
         ci = _CHAIN["ci"]
-        return {"workload": "chain", "recipe": ci.recipe, "R": ci.lcb.R, "C": ci.lcb.C, "sum_L": int(ci.seq_off[-1])}
+        cfg = {"workload": workload, "recipe": ci.recipe, "R": ci.lcb.R, "C": ci.lcb.C, "sum_L": int(ci.seq_off[-1])}
+        if workload == "chain_split":
+            cfg["weights"] = "W_fold and [W_RR; W_CR] prepared once before timing (model preprocessing)"
+        return cfg
     cfg = {"workload": workload, "parts": {}}
     for p in parts:
         x = p.x
@@ -667,6 +734,8 @@ def run_ikbo(args):
     for p in parts:
         if isinstance(p, DcaPart) and args.workload == "chain":
             p.to_device(ikbo, torch, dev, q_dev=parts[1].out)
+        elif isinstance(p, DcaPart) and args.workload == "chain_split":
+            p.to_device(ikbo, torch, dev, q_dev=parts[0].out)
         else:
             p.to_device(ikbo, torch, dev)
     torch.cuda.synchronize()
@@ -799,7 +868,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ikbo", choices=["ikbo", "reference"])
     ap.add_argument("--workload", default="ikbo_step",
-                    choices=["ikbo_step", "lcb", "lcb_block", "fm", "dca", "dca_short", "dca_block", "chain"])
+                    choices=["ikbo_step", "lcb", "lcb_block", "fm", "dca", "dca_short", "dca_block", "chain",
+                             "chain_split"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--no-e2e", action="store_true")

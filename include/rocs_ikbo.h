@@ -338,6 +338,59 @@ ROCS_API size_t rocs_proj_workspace_size(const rocs_proj_args* args);
 ROCS_API int rocs_proj_forward(const rocs_proj_args* args, rocs_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * Split chain: the query projection of the chained block distributed over the IKBO
+ * decomposition (section 3.2 Eq. (12) with section 4.1 Eq. (14); the projection is a plain
+ * linear map):
+ *     Q_i = W_q vec(Y^C_i) = W_q vec(Z_{m_i}) + W_q vec(W_CC X^C_i)
+ *         = q^R_{m_i} + W_fold vec(X^C_i)
+ * with q^R_r = W_q vec(Z_r) computed once per request and W_fold[k, n*d + c] =
+ * sum_o W_q[k, o*d + c] W_CC[o, n] prepared once per model.  Y^C is never written; the
+ * result equals the chain on the exact (unrounded) LCB output up to bf16 rounding of Z_r and
+ * of W_fold.
+ *
+ * rocs_chain_prepare_weights (once per model):
+ *   w_q [n_out, o_c*d], w_rr [o_r, n_r], w_cr [o_c, n_r], w_cc [o_c, n_c]  bf16 in
+ *   w_fold [n_out, n_c*d] bf16 out (fp32 accumulation, one rounding)
+ *   w_rs   [o_r + o_c, n_r] bf16 out: [W_RR; W_CR] stacked
+ *   One launch plus two device-to-device copies on `stream`.
+ * rocs_chain_split_forward (per batch):
+ *   y_req [R, o_r + o_c, d] bf16 out: rows [0, o_r) = Y^R_r, rows [o_r, o_r + o_c) = Z_r
+ *   q     [C, n_out] bf16 out: the candidate queries (input of rocs_dca_forward)
+ *   Shapes as rocs_lcb_forward (ROCS_BF16) with o_r + o_c in place of o_r, n_out % 256 == 0,
+ *   (n_c*d) % 64 == 0.  Workspace rocs_chain_split_workspace_size(); one status header for all
+ *   steps (rocs_read_status).  Three kernel launches plus memsets.
+ * ---------------------------------------------------------------------------------- */
+typedef struct {
+  int64_t n_out, o_r, o_c, n_r, n_c, d;
+  const void* w_q;
+  const void* w_rr;
+  const void* w_cr;
+  const void* w_cc;
+  void* w_fold;
+  void* w_rs;
+} rocs_chain_weights_args;
+
+ROCS_API int rocs_chain_prepare_weights(const rocs_chain_weights_args* args, rocs_stream_t stream);
+
+typedef struct {
+  int64_t R, n_r, n_c, d, o_r, o_c, n_out;
+  const int32_t* cand_off_dev;  /* [R+1] */
+  const int32_t* cand_off_host; /* [R+1] */
+  const void* x_req;  /* [R, n_r, d] */
+  const void* x_cand; /* [C, n_c, d] */
+  const void* w_rs;   /* [o_r + o_c, n_r] from rocs_chain_prepare_weights */
+  const void* w_q;    /* [n_out, o_c*d] */
+  const void* w_fold; /* [n_out, n_c*d] from rocs_chain_prepare_weights */
+  void* y_req;        /* [R, o_r + o_c, d] */
+  void* q;            /* [C, n_out] */
+  void* workspace;
+  size_t workspace_bytes;
+} rocs_chain_split_args;
+
+ROCS_API size_t rocs_chain_split_workspace_size(const rocs_chain_split_args* args);
+ROCS_API int rocs_chain_split_forward(const rocs_chain_split_args* args, rocs_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * Status and introspection
  * ---------------------------------------------------------------------------------- */
 

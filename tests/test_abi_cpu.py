@@ -170,3 +170,32 @@ def test_fm_host_validation(lib):
     assert lib.rocs_pad_cols(fake, 4, 10, 8, fake, 16, 2, None) == 1  # ld_src < cols
     assert lib.rocs_pad_cols(fake + 1, 4, 10, 10, fake, 16, 2, None) == 1  # misaligned
     assert lib.rocs_pad_cols(None, 0, 10, 10, None, 16, 2, None) == 0  # nothing to do
+
+
+def test_chain_split_host_validation(lib):
+    import attention_ikbo_b200 as m
+
+    fake = 0x10000
+    P = ctypes.byref
+    W = m._binding.ChainWeightsArgs
+    assert lib.rocs_chain_prepare_weights(P(W(n_out=256, o_r=128, o_c=128, n_r=256, n_c=64, d=128)), None) == 1
+    S = m._binding.ChainSplitArgs
+
+    def args(off, n_out=256, n_c=64, ws=1 << 22):
+        off = np.asarray(off, np.int32)
+        a = S(R=len(off) - 1, n_r=256, n_c=n_c, d=128, o_r=128, o_c=128, n_out=n_out, cand_off_dev=fake,
+              cand_off_host=off.ctypes.data, x_req=fake, x_cand=fake, w_rs=fake, w_q=fake, w_fold=fake, y_req=fake,
+              q=fake, workspace=fake if ws else None, workspace_bytes=ws)
+        return a, off
+
+    a, k = args([0, 3, 5], n_out=300)
+    assert lib.rocs_chain_split_forward(P(a), None) == 3
+    a, k = args([0, 3, 5], n_c=48)
+    assert lib.rocs_chain_split_forward(P(a), None) == 3
+    a, k = args([0, 3, 2])
+    assert lib.rocs_chain_split_forward(P(a), None) == 2
+    a, k = args([0, 3, 5], ws=100)
+    assert lib.rocs_chain_split_forward(P(a), None) == 6
+    a, k = args([0, 3, 5])
+    # LCB workspace (header, flags, Z fp32 2 x 128 x 128) padded to 256, then q^R fp32 2 x 256
+    assert lib.rocs_chain_split_workspace_size(P(a)) == 256 + 256 + 2 * 128 * 128 * 4 + 2 * 256 * 4
