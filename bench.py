@@ -600,16 +600,25 @@ def kernel_sha(kernel):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel, units):
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+def part_signature(p):
+    """The inputs a part's ncu capture was taken on: name, kernel, sizes and recipe."""
+    x = getattr(p, "x", None) or getattr(p, "ci", None)
+    desc = {"name": p.name, "kernel": p.kernel, "units": p.units,
+            "recipe": getattr(x, "recipe", "") or getattr(getattr(x, "lcb", None), "recipe", "")}
+    return hashlib.sha256(json.dumps(desc, sort_keys=True).encode()).hexdigest()[:16]
+
+
+def ncu_traffic(p):
+    """DRAM bytes per launch of the part's kernel from the committed ncu summary: only if the capture was
+    taken on the current kernel source and on the same inputs (traffic per candidate is workload-specific)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        d = json.load(f).get(kernel)
-    if not d or d.get("src_sha") != kernel_sha(kernel):
+        d = json.load(f).get(p.name)
+    if not d or d.get("src_sha") != kernel_sha(p.kernel) or d.get("inputs") != part_signature(p):
         return None
-    return d["dram_bytes_per_unit"] * units
+    return d["dram_bytes_per_unit"] * p.units
 
 
 class ClockSampler:
@@ -833,7 +842,7 @@ def run_ikbo(args):
         else:
             ach, peak, unit = p.flops() / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
         rf = {"kernel": p.name, "bound": p.bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
-              "traffic": ncu_traffic(p.kernel, p.units), "peak_source": f"{peak_src} (burst)"}
+              "traffic": ncu_traffic(p), "peak_source": f"{peak_src} (burst)"}
         rooflines.append(rf)
         part_rows.append({"name": p.name, "ms": ms, "tflops": p.flops() / sec / 1e12, "gbs": p.bytes() / sec / 1e9,
                           "candidates_per_s": p.units / sec, "algorithmic_flops": p.flops(),
