@@ -18,6 +18,8 @@ Operations ("ROCS: Request-Oriented Compute Sharing ...", arXiv:2607.27744):
     stored once per request (section 4.3).
   * :func:`rocs_dca_block_forward` -- both query groups of Eq. (13) with the K/V projections
     done once per request (section 4.1).
+  * :func:`rocs_lcb_forward_host` / :func:`rocs_dca_forward_host` -- the same on batches in pinned
+    host memory, copies and compute pipelined over request chunks.
   * :func:`rocs_proj_forward` -- linear query projection of the chained block (Eq. 12).
   * :func:`rocs_chain_split_forward` / :func:`chain_split_forward` -- the chain with the projection
     split over the IKBO decomposition (request term once per request, W_q folded with W_CC by
@@ -39,11 +41,13 @@ from ._binding import (  # noqa: F401
     rocs_dca_block_forward,
     rocs_dca_forward,
     rocs_dca_forward_expand,
+    rocs_dca_forward_host,
     rocs_fm_forward,
     rocs_lcb_block_forward,
     rocs_lcb_forward,
     rocs_lcb_forward_expand,
     rocs_lcb_forward_fault_injection,
+    rocs_lcb_forward_host,
     rocs_lcb_forward_noalloc,
     rocs_pad_cols,
     rocs_proj_forward,

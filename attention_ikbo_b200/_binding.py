@@ -114,6 +114,14 @@ def load_library():
                            ("rocs_read_status", [_vp, _vp, P(_i32), P(_i32)])]:
             getattr(lib, name).restype = ctypes.c_int
             getattr(lib, name).argtypes = argt
+        for name, argt in [("rocs_lcb_host_staging_size", [P(LcbArgs), _i64]),
+                           ("rocs_dca_host_staging_size", [P(DcaArgs), _i64])]:
+            getattr(lib, name).restype = _sz
+            getattr(lib, name).argtypes = argt
+        lib.rocs_lcb_forward_host.restype = ctypes.c_int
+        lib.rocs_lcb_forward_host.argtypes = [P(LcbArgs), _i64, _vp, _sz, _vp]
+        lib.rocs_dca_forward_host.restype = ctypes.c_int
+        lib.rocs_dca_forward_host.argtypes = [P(DcaArgs), _i64, _vp, _sz, _vp]
         lib.rocs_align_cols.restype = _i64
         lib.rocs_align_cols.argtypes = [_i64, _i64]
         lib.rocs_status_string.restype = ctypes.c_char_p
@@ -532,3 +540,76 @@ def chain_split_forward(x_req, x_cand, w_rs, w_q, w_fold, cand_off, o_r, k_t, v_
     o, lse = rocs_dca_forward(q.view(C, heads, head_dim), k_t, v_t, cand_off, seq_off, 1, scale,
                               workspace=ws.get("dca"), stream=stream)
     return y_req, q, o, lse
+
+
+def _host_tensor(t, what):
+    if t.is_cuda or not t.is_contiguous() or not t.is_pinned():
+        raise RocsError(1, f"{what} must be a contiguous pinned host tensor")
+
+
+def rocs_lcb_forward_host(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req=None, y_cand=None, chunks=8,
+                          staging=None, stream=None):
+    """IKBO-LCB on a host-resident batch: pinned host ``x_req``/``x_cand`` in, pinned host ``y_req``/``y_cand``
+    out, device weights; copies and compute pipelined over request chunks (see the header)."""
+    lib = load_library()
+    dev = w_rr.device
+    off_d, off_h = _offsets(cand_off, dev)
+    R, n_r, d = x_req.shape
+    C = int(off_h[-1])
+    n_c, o_r, o_c = x_cand.shape[1], w_rr.shape[0], w_cc.shape[0]
+    dt = x_req.dtype
+    if y_req is None:
+        y_req = torch.empty((R, o_r, d), dtype=dt, pin_memory=True)
+    if y_cand is None:
+        y_cand = torch.empty((C, o_c, d), dtype=dt, pin_memory=True)
+    for t, n in ((x_req, "x_req"), (x_cand, "x_cand"), (y_req, "y_req"), (y_cand, "y_cand")):
+        _host_tensor(t, n)
+    for t in (w_rr, w_cr, w_cc):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == dt):
+            raise RocsError(1, "LCB weights must be contiguous CUDA tensors of the batch dtype")
+    a = LcbArgs(R=R, n_r=n_r, n_c=n_c, d=d, o_r=o_r, o_c=o_c, dtype={torch.float32: ROCS_F32, torch.bfloat16: ROCS_BF16}[dt],
+                cand_off_dev=off_d.data_ptr(), cand_off_host=off_h.ctypes.data, x_req=x_req.data_ptr(),
+                x_cand=x_cand.data_ptr() if C else None, w_rr=w_rr.data_ptr(), w_cr=w_cr.data_ptr(),
+                w_cc=w_cc.data_ptr(), y_req=y_req.data_ptr(), y_cand=y_cand.data_ptr() if C else None)
+    nbytes = lib.rocs_lcb_host_staging_size(ctypes.byref(a), int(chunks))
+    if nbytes == 0:
+        _check(lib.rocs_lcb_forward_host(ctypes.byref(a), int(chunks), None, 0, _stream(stream)), "rocs_lcb_forward_host")
+    st = _workspace(nbytes, dev, staging)
+    _check(lib.rocs_lcb_forward_host(ctypes.byref(a), int(chunks), _ptr(st), st.numel(), _stream(stream)),
+           "rocs_lcb_forward_host")
+    rocs_lcb_forward_host.last_staging = st
+    rocs_lcb_forward_host.keep = (off_d, off_h)
+    return y_req, y_cand
+
+
+def rocs_dca_forward_host(q_t, k_t, v_t, cand_off, seq_off, q_tokens, scale, o=None, lse=True, device="cuda",
+                          chunks=4, staging=None, stream=None):
+    """IKBO-DCA on a host-resident batch: pinned host Q/K/V in, pinned host O (and LSE) out."""
+    lib = load_library()
+    dev = torch.device(device)
+    co_d, co_h = _offsets(cand_off, dev)
+    so_d, so_h = _offsets(seq_off, dev)
+    R = len(co_h) - 1
+    H, dh = k_t.shape[1], k_t.shape[2]
+    if o is None:
+        o = torch.empty(q_t.shape, dtype=torch.bfloat16, pin_memory=True)
+    if lse is True:
+        lse = torch.empty(q_t.shape[:2], dtype=torch.float32, pin_memory=True)
+    elif lse is False:
+        lse = None
+    for t, n in ((q_t, "q"), (k_t, "k"), (v_t, "v"), (o, "o")) + (((lse, "lse"),) if lse is not None else ()):
+        _host_tensor(t, n)
+    a = DcaArgs(R=R, q=q_tokens, H=H, dh=dh, scale=float(scale), cand_off_dev=co_d.data_ptr(),
+                cand_off_host=co_h.ctypes.data, seq_off_dev=so_d.data_ptr(), seq_off_host=so_h.ctypes.data,
+                q_ptr=q_t.data_ptr() if q_t.numel() else None, k_ptr=k_t.data_ptr() if k_t.numel() else None,
+                v_ptr=v_t.data_ptr() if v_t.numel() else None, o_ptr=o.data_ptr() if o.numel() else None,
+                lse_ptr=lse.data_ptr() if lse is not None else None)
+    nbytes = lib.rocs_dca_host_staging_size(ctypes.byref(a), int(chunks))
+    if nbytes == 0:
+        _check(lib.rocs_dca_forward_host(ctypes.byref(a), int(chunks), None, 0, _stream(stream)), "rocs_dca_forward_host")
+    st = _workspace(nbytes, dev, staging)
+    _check(lib.rocs_dca_forward_host(ctypes.byref(a), int(chunks), _ptr(st), st.numel(), _stream(stream)),
+           "rocs_dca_forward_host")
+    rocs_dca_forward_host.last_staging = st
+    rocs_dca_forward_host.keep = (co_d, co_h, so_d, so_h)
+    return o, lse

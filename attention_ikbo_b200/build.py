@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "librocs_ikbo.so")
 SOURCES = ["rocs_abi.cu", "lcb_sm100.cu", "lcb_f32.cu", "dca_sm100.cu", "proj_sm100.cu", "expand.cu", "lcb_noalloc.cu",
-           "fm_sm100.cu"]
+           "fm_sm100.cu", "host_pipeline.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
          "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

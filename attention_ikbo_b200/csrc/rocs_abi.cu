@@ -342,6 +342,7 @@ int dca_run_ext(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, W
   return dca_run(a, C, T, n_units, hdr, body, st, launches);
 }
 size_t dca_body_bytes_ext(int64_t R, int64_t n_units) { return dca_body(R, n_units).body; }
+int64_t dca_units_ext(const rocs_dca_args* a) { return dca_units(a); }
 void set_last_launches(int n) { g_last_launches = n; }
 }  // namespace rocs
 

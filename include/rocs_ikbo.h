@@ -391,6 +391,31 @@ ROCS_API size_t rocs_chain_split_workspace_size(const rocs_chain_split_args* arg
 ROCS_API int rocs_chain_split_forward(const rocs_chain_split_args* args, rocs_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * Host-resident batches (no counterpart in the paper: the serving path of a batch that lives in
+ * host memory).  The same operations as rocs_lcb_forward / rocs_dca_forward, but the batch
+ * tensors are HOST pointers (pinned memory, so the copies run asynchronously):
+ *   LCB: x_req, x_cand in; y_req, y_cand out (host).  Weights w_* and cand_off_dev stay on the
+ *        device; cand_off_host as usual.
+ *   DCA: q_ptr, k_ptr, v_ptr in; o_ptr, lse_ptr (or NULL) out (host); cand_off_dev, seq_off_dev
+ *        on the device; kv_ld must be 0 (or H*dh).
+ * The batch is cut into `chunks` groups of whole requests of about equal bytes; chunk c is computed
+ * while chunk c+1 is copied in and chunk c-1 copied out, through two device staging slots held in
+ * `staging` (>= rocs_*_host_staging_size(args, chunks) bytes, 256-byte aligned, caller-owned; the
+ * args' workspace fields are ignored).  Copies and kernels run on three streams the library creates
+ * once per device and keeps; `stream` waits for the whole call, so work enqueued on it afterwards
+ * (e.g. a host read of the outputs after a synchronize) sees every output.  Device status of all
+ * chunks is kept in the first 256 bytes of `staging` (rocs_read_status(staging, ...)).  Errors as
+ * for the device entry points; a host error returned after some chunks were enqueued leaves the
+ * outputs of those chunks to complete.
+ * ---------------------------------------------------------------------------------- */
+ROCS_API size_t rocs_lcb_host_staging_size(const rocs_lcb_args* args, int64_t chunks);
+ROCS_API int rocs_lcb_forward_host(const rocs_lcb_args* args, int64_t chunks, void* staging, size_t staging_bytes,
+                                   rocs_stream_t stream);
+ROCS_API size_t rocs_dca_host_staging_size(const rocs_dca_args* args, int64_t chunks);
+ROCS_API int rocs_dca_forward_host(const rocs_dca_args* args, int64_t chunks, void* staging, size_t staging_bytes,
+                                   rocs_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * Status and introspection
  * ---------------------------------------------------------------------------------- */
 

@@ -199,3 +199,18 @@ def test_chain_split_host_validation(lib):
     a, k = args([0, 3, 5])
     # LCB workspace (header, flags, Z fp32 2 x 128 x 128) padded to 256, then q^R fp32 2 x 256
     assert lib.rocs_chain_split_workspace_size(P(a)) == 256 + 256 + 2 * 128 * 128 * 4 + 2 * 256 * 4
+
+
+def test_host_pipeline_host_validation(lib):
+    import attention_ikbo_b200 as m
+
+    a, keep = _lcb_args(m, [0, 3, 6])
+    P = ctypes.byref
+    assert lib.rocs_lcb_host_staging_size(P(a), 0) == 0  # chunks >= 1
+    need = lib.rocs_lcb_host_staging_size(P(a), 2)
+    assert need > 256
+    assert lib.rocs_lcb_forward_host(P(a), 0, 0x10000, need, None) == 1
+    assert lib.rocs_lcb_forward_host(P(a), 2, 0x10000, need - 1, None) == 6
+    assert lib.rocs_lcb_forward_host(P(a), 2, None, need, None) == 6
+    bad, keep2 = _lcb_args(m, [0, 3, 2])
+    assert lib.rocs_lcb_forward_host(P(bad), 2, 0x10000, need, None) == 2
