@@ -171,12 +171,19 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       uint32_t rs = 0, rph = 0, ws_ = 0, wph = 0, qeph[2] = {0, 0};
       int n_issued = 0;
       bool ok = true;
-      auto load_kv = [&](const CUtensorMap* tm, int y, int x0) -> bool {
+      // the ring holds under two steps of K/V; tiles kPrefetch steps ahead are started towards L2 so that
+      // the ring's loads find them there (the K/V of all requests need not fit in L2)
+      constexpr int kPrefetch = 4;
+      auto load_kv = [&](const CUtensorMap* tm, int y, int x0, int y_end) -> bool {
         if (!mbar_wait(&ring_empty[rs], rph ^ 1, ctl, 501)) return false;
         uint8_t* slot = s_ring + rs * L::kTile;
         mbar_arrive_expect_tx(&ring_full[rs], L::kTile);
 #pragma unroll
         for (int cc = 0; cc < DH / 64; ++cc) tma_load_2d(slot + cc * (BM * 128), tm, &ring_full[rs], x0 + cc * 64, y);
+        if (y + kPrefetch * BN < y_end) {
+#pragma unroll
+          for (int cc = 0; cc < DH / 64; ++cc) tma_prefetch_l2_2d(tm, x0 + cc * 64, y + kPrefetch * BN);
+        }
         ++n_issued;
         if (++rs == kRing) { rs = 0; rph ^= 1; }
         return true;
@@ -202,13 +209,21 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
                         w.qbase + w.row0 + x * BM);
         }
         if (!ok) break;
-        // K/V in the order the MMA issuer consumes them: K0, (K1, V0), (K2, V1), ..., V_last
-        ok = load_kv(&p.tm_k, w.s0, x0);
+        // K/V in the order the MMA issuer consumes them: K0, (K1, V0), (K2, V1), ..., V_last; the first
+        // kPrefetch tiles of each are started towards L2 before the ring loads begin
+        const int y_end = w.s0 + w.L;
+        for (int j = 0; j < kPrefetch && j < w.nkv; ++j)
+#pragma unroll
+          for (int cc = 0; cc < DH / 64; ++cc) {
+            tma_prefetch_l2_2d(&p.tm_k, x0 + cc * 64, w.s0 + j * BN);
+            tma_prefetch_l2_2d(&p.tm_v, x0 + cc * 64, w.s0 + j * BN);
+          }
+        ok = load_kv(&p.tm_k, w.s0, x0, y_end);
         for (int j = 1; ok && j < w.nkv; ++j) {
-          ok = load_kv(&p.tm_k, w.s0 + j * BN, x0);
-          if (ok) ok = load_kv(&p.tm_v, w.s0 + (j - 1) * BN, x0);
+          ok = load_kv(&p.tm_k, w.s0 + j * BN, x0, y_end);
+          if (ok) ok = load_kv(&p.tm_v, w.s0 + (j - 1) * BN, x0, y_end);
         }
-        if (ok) ok = load_kv(&p.tm_v, w.s0 + (w.nkv - 1) * BN, x0);
+        if (ok) ok = load_kv(&p.tm_v, w.s0 + (w.nkv - 1) * BN, x0, y_end);
       }
       if (!ok) {
         for (int k = n_issued > kRing ? n_issued - kRing : 0; k < n_issued; ++k)
@@ -361,56 +376,83 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
             for (int k = 0; k < 32; ++k)
               if (c4 * 32 + k >= kvalid) sv[c4][k] = __float_as_uint(-INFINITY);
         }
+        // P = exp2(c S - m) written over S.  From the second tile on, the exponentials use the running
+        // max m_used at once and the tile's own row max is computed alongside them (off the critical
+        // path); if some row's max exceeds m_used by more than 2^8 the tile is redone with the new max
+        // after rescaling O (rare: the max settles after the first tiles).  Until then P <= 2^8, which
+        // bf16 and the fp32 sums hold.
+        uint64_t ls0, ls1;
         float mq[8];
+        auto exps_pass = [&](bool with_max) {
+          uint64_t c2, nm2;
+          asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(c));
+          asm("mov.b64 %0, {%1, %1};" : "=l"(nm2) : "f"(-m_used));
+          ls0 = 0;
+          ls1 = 0;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mq[k] = -INFINITY;
+          for (int k = 0; k < 8; ++k) mq[k] = -INFINITY;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            float y;
-            asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(mq[k & 7]), "f"(__uint_as_float(sv[c4][2 * k])), "f"(__uint_as_float(sv[c4][2 * k + 1])));
-            mq[k & 7] = y;
+            for (int k = 0; k < 16; ++k) {
+              if (with_max) {
+                float y;
+                asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(mq[k & 7]), "f"(__uint_as_float(sv[c4][2 * k])),
+                    "f"(__uint_as_float(sv[c4][2 * k + 1])));
+                mq[k & 7] = y;
+              }
+              uint64_t sp, xp, ep;
+              asm("mov.b64 %0, {%1, %2};" : "=l"(sp) : "r"(sv[c4][2 * k]), "r"(sv[c4][2 * k + 1]));
+              asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(xp) : "l"(sp), "l"(c2), "l"(nm2));
+              float x0, x1;
+              asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(xp));
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              asm("mov.b64 %0, {%1, %2};" : "=l"(ep) : "f"(p0), "f"(p1));
+              if (k & 1) asm("add.f32x2 %0, %1, %2;" : "=l"(ls1) : "l"(ls1), "l"(ep));
+              else asm("add.f32x2 %0, %1, %2;" : "=l"(ls0) : "l"(ls0), "l"(ep));
+              pk[k] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(s_addr + c4 * 16, pk);
           }
-        const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
-        const float mxs = mx * c;
-        if (j == 0) {
-          m_used = mxs;
-        } else if (__any_sync(0xffffffffu, mxs > m_used + 8.0f)) {
-          const float m_new = fmaxf(m_used, mxs);
-          const float f = ex2(m_used - m_new);
-          l *= f;
+        };
+        auto row_max = [&]() {
+          return fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
+        };
+        if (j == 0) {  // first tile: the max first
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mq[k] = -INFINITY;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              float y;
+              asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(mq[k & 7]), "f"(__uint_as_float(sv[c4][2 * k])),
+                  "f"(__uint_as_float(sv[c4][2 * k + 1])));
+              mq[k & 7] = y;
+            }
+          m_used = row_max() * c;
+          exps_pass(false);
+        } else {
+          exps_pass(true);
+          const float mxs = row_max() * c;
+          if (__any_sync(0xffffffffu, mxs > m_used + 8.0f)) {  // rare: rescale O, redo the tile
+            const float m_new = fmaxf(m_used, mxs);
+            const float f = ex2(m_used - m_new);
+            l *= f;
+            tmem_st_wait();
 #pragma unroll 1
-          for (int cc = 0; cc < DH / 32; ++cc) {
-            uint32_t ov[32];
-            tmem_ld32(o_addr + cc * 32, ov);
-            tmem_ld_wait();
+            for (int cc = 0; cc < DH / 32; ++cc) {
+              uint32_t ov[32];
+              tmem_ld32(o_addr + cc * 32, ov);
+              tmem_ld_wait();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-            tmem_st32(o_addr + cc * 32, ov);
+              for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+              tmem_st32(o_addr + cc * 32, ov);
+            }
+            m_used = m_new;
+            exps_pass(false);
           }
-          m_used = m_new;
-        }
-        uint64_t c2, nm2, ls0 = 0, ls1 = 0;
-        asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(c));
-        asm("mov.b64 %0, {%1, %1};" : "=l"(nm2) : "f"(-m_used));
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            uint64_t sp, xp, ep;
-            asm("mov.b64 %0, {%1, %2};" : "=l"(sp) : "r"(sv[c4][2 * k]), "r"(sv[c4][2 * k + 1]));
-            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(xp) : "l"(sp), "l"(c2), "l"(nm2));
-            float x0, x1;
-            asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(xp));
-            const float p0 = ex2(x0), p1 = ex2(x1);
-            asm("mov.b64 %0, {%1, %2};" : "=l"(ep) : "f"(p0), "f"(p1));
-            if (k & 1) asm("add.f32x2 %0, %1, %2;" : "=l"(ls1) : "l"(ls1), "l"(ep));
-            else asm("add.f32x2 %0, %1, %2;" : "=l"(ls0) : "l"(ls0), "l"(ep));
-            pk[k] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(s_addr + c4 * 16, pk);
         }
         float la, lb, lc, ld;
         asm("mov.b64 {%0, %1}, %2;" : "=f"(la), "=f"(lb) : "l"(ls0));
