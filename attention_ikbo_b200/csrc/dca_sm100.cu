@@ -171,19 +171,12 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       uint32_t rs = 0, rph = 0, ws_ = 0, wph = 0, qeph[2] = {0, 0};
       int n_issued = 0;
       bool ok = true;
-      // the ring holds under two steps of K/V; tiles kPrefetch steps ahead are started towards L2 so that
-      // the ring's loads find them there (the K/V of all requests need not fit in L2)
-      constexpr int kPrefetch = 4;
-      auto load_kv = [&](const CUtensorMap* tm, int y, int x0, int y_end) -> bool {
+      auto load_kv = [&](const CUtensorMap* tm, int y, int x0) -> bool {
         if (!mbar_wait(&ring_empty[rs], rph ^ 1, ctl, 501)) return false;
         uint8_t* slot = s_ring + rs * L::kTile;
         mbar_arrive_expect_tx(&ring_full[rs], L::kTile);
 #pragma unroll
         for (int cc = 0; cc < DH / 64; ++cc) tma_load_2d(slot + cc * (BM * 128), tm, &ring_full[rs], x0 + cc * 64, y);
-        if (y + kPrefetch * BN < y_end) {
-#pragma unroll
-          for (int cc = 0; cc < DH / 64; ++cc) tma_prefetch_l2_2d(tm, x0 + cc * 64, y + kPrefetch * BN);
-        }
         ++n_issued;
         if (++rs == kRing) { rs = 0; rph ^= 1; }
         return true;
@@ -209,21 +202,13 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
                         w.qbase + w.row0 + x * BM);
         }
         if (!ok) break;
-        // K/V in the order the MMA issuer consumes them: K0, (K1, V0), (K2, V1), ..., V_last; the first
-        // kPrefetch tiles of each are started towards L2 before the ring loads begin
-        const int y_end = w.s0 + w.L;
-        for (int j = 0; j < kPrefetch && j < w.nkv; ++j)
-#pragma unroll
-          for (int cc = 0; cc < DH / 64; ++cc) {
-            tma_prefetch_l2_2d(&p.tm_k, x0 + cc * 64, w.s0 + j * BN);
-            tma_prefetch_l2_2d(&p.tm_v, x0 + cc * 64, w.s0 + j * BN);
-          }
-        ok = load_kv(&p.tm_k, w.s0, x0, y_end);
+        // K/V in the order the MMA issuer consumes them: K0, (K1, V0), (K2, V1), ..., V_last
+        ok = load_kv(&p.tm_k, w.s0, x0);
         for (int j = 1; ok && j < w.nkv; ++j) {
-          ok = load_kv(&p.tm_k, w.s0 + j * BN, x0, y_end);
-          if (ok) ok = load_kv(&p.tm_v, w.s0 + (j - 1) * BN, x0, y_end);
+          ok = load_kv(&p.tm_k, w.s0 + j * BN, x0);
+          if (ok) ok = load_kv(&p.tm_v, w.s0 + (j - 1) * BN, x0);
         }
-        if (ok) ok = load_kv(&p.tm_v, w.s0 + (w.nkv - 1) * BN, x0, y_end);
+        if (ok) ok = load_kv(&p.tm_v, w.s0 + (w.nkv - 1) * BN, x0);
       }
       if (!ok) {
         for (int k = n_issued > kRing ? n_issued - kRing : 0; k < n_issued; ++k)
