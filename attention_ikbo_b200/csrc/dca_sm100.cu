@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         return true;
       };
       while (ok) {
-        const int t = atomicAdd(&p.ws->counter, 1);
+        const int t = atomicAdd(p.ticket, 1);
         const int item = t < p.n_units ? t : -1;
         if (!mbar_wait(&wq_empty[ws_], wph ^ 1, ctl, 502)) { ok = false; break; }
         s_wq[ws_] = item;
@@ -544,7 +544,7 @@ __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
     run += p.H * nb;
   }
   if (t == T - 1 && s_part[T - 1] != p.max_units) record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 802);
-  if (t == 0) p.ws->counter = 0;
+  if (t == 0) *p.ticket = 0;
 }
 
 cudaError_t launch_dca_schedule(const DcaSchedParams& p, cudaStream_t st) {

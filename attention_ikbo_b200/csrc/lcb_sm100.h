@@ -45,6 +45,7 @@ struct DcaParams {
   const int32_t* cand_off;
   const int32_t* seq_off;
   const int4* units;  // work-unit table {r, h, row0, 0}
+  int* ticket;        // work-unit counter (zeroed by the schedule kernel)
   __nv_bfloat16* o;
   float* lse;
   WsHeader* ws;
@@ -60,6 +61,7 @@ struct DcaSchedParams {
   int* scratch;  // 3R+1 ints
   int4* units;
   WsHeader* ws;
+  int* ticket;  // the counter the attention kernel claims units from (zeroed here)
   int R, q, H, rows_per_unit, max_units;
 };
 cudaError_t launch_dca_schedule(const DcaSchedParams& p, cudaStream_t st);

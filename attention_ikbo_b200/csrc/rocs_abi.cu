@@ -3,6 +3,7 @@
 // No entry point allocates or frees memory or synchronises a stream (except
 // rocs_read_status, whose job is to synchronise and read).
 #include <cmath>
+#include <mutex>
 #include <cstring>
 
 #include "lcb_sm100.h"
@@ -16,6 +17,30 @@ using namespace rocs;
 namespace {
 
 thread_local int g_last_launches = 0;
+
+// A second stream per device (created on first use, kept for the process) with a fork and a join
+// event, for launches that run beside the caller's stream inside one call.
+struct AuxStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool ok = false;
+};
+AuxStream* aux_stream_for_current_device() {
+  static std::mutex mu;
+  static AuxStream aux[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  AuxStream& x = aux[dev];
+  if (!x.ok) {
+    if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    x.ok = true;
+  }
+  return &x;
+}
 
 int sm_count() {
   int dev = 0, n = 148;
@@ -280,8 +305,10 @@ int dca_validate(const rocs_dca_args* a, int64_t* C, int64_t* T) {
   return ROCS_OK;
 }
 
+// ticket: the work counter of this launch (default: the header's); two launches that run at the same
+// time on one header use different counters
 int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHeader* hdr, uint8_t* w,
-            cudaStream_t st, int* launches, bool reset_header = true) {
+            cudaStream_t st, int* launches, bool reset_header = true, int* ticket = nullptr) {
   const DcaLayout L = dca_body(a->R, n_units);
   if (n_units >= (int64_t(1) << 31)) return ROCS_ERR_UNSUPPORTED;
   if (reset_header && cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return ROCS_ERR_CUDA;
@@ -292,6 +319,7 @@ int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHea
   sp.scratch = reinterpret_cast<int*>(w + L.scratch);
   sp.units = reinterpret_cast<int4*>(w + L.units);
   sp.ws = hdr;
+  sp.ticket = ticket ? ticket : &hdr->counter;
   sp.R = (int)a->R;
   sp.q = (int)a->q;
   sp.H = (int)a->H;
@@ -316,6 +344,7 @@ int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHea
   p.o = static_cast<__nv_bfloat16*>(a->o_ptr);
   p.lse = a->lse_ptr;
   p.ws = sp.ws;
+  p.ticket = sp.ticket;
   p.R = (int)a->R;
   p.q = (int)a->q;
   p.H = (int)a->H;
@@ -501,6 +530,12 @@ extern "C" int rocs_dca_block_forward(const rocs_dca_block_args* a, rocs_stream_
   int32_t* ident = reinterpret_cast<int32_t*>(w + L.ident);
   if (launch_ident(ident, (int)a->R, st) != cudaSuccess) return ROCS_ERR_CUDA;
   ++launches;
+  // The request group (one unit per request and head, few of them, each as long as a request's key
+  // sequence) runs on a second stream at the same time as the candidate group: launched first, it
+  // takes its SMs before the persistent candidate kernel fills the rest, instead of forming a tail.
+  AuxStream* aux = aux_stream_for_current_device();
+  if (!aux || cudaEventRecord(aux->fork, st) != cudaSuccess || cudaStreamWaitEvent(aux->s, aux->fork, 0) != cudaSuccess)
+    return ROCS_ERR_CUDA;
   rocs_dca_args d;
   std::memset(&d, 0, sizeof(d));
   d.R = a->R;
@@ -510,7 +545,6 @@ extern "C" int rocs_dca_block_forward(const rocs_dca_block_args* a, rocs_stream_
   d.seq_off_dev = a->seq_off_dev;
   d.seq_off_host = a->seq_off_host;
   d.kv_ld = 4 * hd;
-  // candidate group (IKBO: K/V at batch B_r, m_i resolved in the kernel)
   d.q = a->q;
   d.cand_off_dev = a->cand_off_dev;
   d.cand_off_host = a->cand_off_host;
@@ -520,23 +554,28 @@ extern "C" int rocs_dca_block_forward(const rocs_dca_block_args* a, rocs_stream_
   d.o_ptr = a->o_c;
   d.lse_ptr = a->lse_c;
   int n = 0;
+  // request group: every request is its own single "candidate" with q_r query tokens
+  rocs_dca_args dr = d;
+  dr.q = a->q_req;
+  dr.cand_off_dev = ident;
+  dr.cand_off_host = nullptr;
+  dr.q_ptr = a->q_r;
+  dr.k_ptr = kv + 2 * hd * 2;
+  dr.v_ptr = kv + 3 * hd * 2;
+  dr.o_ptr = a->o_r;
+  dr.lse_ptr = a->lse_r;
+  rc = dca_run(&dr, a->R, L.T, L.units_r, hdr, w + L.body_r, aux->s, &n, false, &hdr->counter2);
+  if (rc) return rc;
+  launches += n;
+  if (cudaEventRecord(aux->join, aux->s) != cudaSuccess) return ROCS_ERR_CUDA;
+  // candidate group (IKBO: K/V at batch B_r, m_i resolved in the kernel)
   if (L.C > 0) {
     rc = dca_run(&d, L.C, L.T, L.units_c, hdr, w + L.body_c, st, &n, false);
     if (rc) return rc;
     launches += n;
   }
-  // request group: every request is its own single "candidate" with q_r query tokens
-  d.q = a->q_req;
-  d.cand_off_dev = ident;
-  d.cand_off_host = nullptr;
-  d.q_ptr = a->q_r;
-  d.k_ptr = kv + 2 * hd * 2;
-  d.v_ptr = kv + 3 * hd * 2;
-  d.o_ptr = a->o_r;
-  d.lse_ptr = a->lse_r;
-  rc = dca_run(&d, a->R, L.T, L.units_r, hdr, w + L.body_r, st, &n, false);
-  if (rc) return rc;
-  g_last_launches = launches + n;
+  if (cudaStreamWaitEvent(st, aux->join, 0) != cudaSuccess) return ROCS_ERR_CUDA;
+  g_last_launches = launches;
   return ROCS_OK;
 }
 
