@@ -832,12 +832,21 @@ def run_ikbo(args):
         def host_capable(p):
             return hasattr(p, "host_run") and not (isinstance(p, DcaPart) and len(p.h_in) != 3)
 
+        part_streams = [torch.cuda.Stream(device=dev) for _ in parts]
+
         def e2e_step():
             hi = ho = 0
             if all(host_capable(p) for p in parts):
-                for p in parts:
-                    a, b = p.host_run(ikbo)
+                # independent batches: each part's host call on its own stream, so one batch's copies
+                # and compute run while another's are still in flight; the timing stream joins them
+                cur = torch.cuda.current_stream()
+                for p, ps in zip(parts, part_streams):
+                    ps.wait_stream(cur)
+                    with torch.cuda.stream(ps):
+                        a, b = p.host_run(ikbo)
                     hi, ho = hi + a, ho + b
+                for ps in part_streams:
+                    cur.wait_stream(ps)
                 return hi, ho
             for p in parts:
                 hi += p.h2d()
