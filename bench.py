@@ -194,6 +194,25 @@ class LcbBlockPart(LcbPart):
         return time.perf_counter() - t0, len(sel) / x.C
 
 
+class LcbExpandPart(LcbPart):
+    """Explicit-expand baseline on the LCB inputs: X^R materialised per candidate, then the same
+    kernel with the identity map (rocs_lcb_forward_expand).  Reported on the IKBO algorithmic work."""
+    kernel = "lcb"
+
+    def __init__(self, x, name="lcb_expand"):
+        super().__init__(x, name)
+
+    def to_device(self, ikbo, torch, dev):
+        super().to_device(ikbo, torch, dev)
+        ikbo.rocs_lcb_forward(*self.d_in, *self.d_w, self.off, self.y_req, self.y_cand, expand=True)
+        self.ws = ikbo.rocs_lcb_forward.last_workspace
+
+    def run(self, ikbo):
+        ikbo.rocs_lcb_forward(*self.d_in, *self.d_w, self.off, self.y_req, self.y_cand, workspace=self.ws,
+                              expand=True)
+        return ikbo.last_launch_count()
+
+
 class FmPart(Part):
     """IKBO masked FM (Eq. 10), rows in the aligned (padded) layout."""
     bound, kernel = "hbm", "fm"
@@ -335,6 +354,28 @@ class DcaPart(Part):
         t0 = time.perf_counter()
         oracle.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, x.v_t, x.q, x.scale, sel_cand=sel)
         return time.perf_counter() - t0, frac
+
+
+class DcaExpandPart(DcaPart):
+    """Explicit-expand baseline on the DCA inputs: K/V copied per candidate in chunks of 1024
+    candidates, each chunk attended with the identity map (rocs_dca_forward_expand)."""
+    chunk = 1024
+
+    def __init__(self, x, name="dca_expand"):
+        super().__init__(x, name)
+
+    def to_device(self, ikbo, torch, dev, q_dev=None):
+        super().to_device(ikbo, torch, dev, q_dev)
+        x = self.x
+        ikbo.rocs_dca_forward(self.q_view(), self.k_dev, self.v_dev, self.coff, self.soff, x.q, x.scale, self.o,
+                              self.lse, expand_chunk=self.chunk)
+        self.ws = ikbo.rocs_dca_forward.last_workspace
+
+    def run(self, ikbo):
+        x = self.x
+        ikbo.rocs_dca_forward(self.q_view(), self.k_dev, self.v_dev, self.coff, self.soff, x.q, x.scale, self.o,
+                              self.lse, workspace=self.ws, expand_chunk=self.chunk)
+        return ikbo.last_launch_count()
 
 
 class DcaBlockPart(Part):
@@ -565,6 +606,10 @@ def make_parts(workload):
         return [LcbBlockPart(ri.lcb_block())]
     if workload == "fm":
         return [FmPart(ri.fm_bf16())]
+    if workload == "lcb_expand":
+        return [LcbExpandPart(ri.lcb_bf16())]
+    if workload == "dca_expand":
+        return [DcaExpandPart(ri.dca_long())]
     if workload == "chain":
         ci = ri.chain()
         lcb = LcbPart(ci.lcb, "chain_lcb")
@@ -925,7 +970,7 @@ def main():
     ap.add_argument("--impl", default="ikbo", choices=["ikbo", "reference"])
     ap.add_argument("--workload", default="ikbo_step",
                     choices=["ikbo_step", "lcb", "lcb_block", "fm", "dca", "dca_short", "dca_block", "chain",
-                             "chain_split"])
+                             "chain_split", "lcb_expand", "dca_expand"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--no-e2e", action="store_true")
