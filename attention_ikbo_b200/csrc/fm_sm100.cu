@@ -14,8 +14,10 @@
 // followed by zeros up to ld_cand, Y^R rows n_r values and zeros up to ld_req, where the leading
 // dimensions are 16-byte multiples, so every row moves by TMA even when n_r + n_c is not.
 //
-// Roles: warps 0-3 epilogue (TMEM -> bf16 rows in the store's swizzled staging -> TMA stores), warp 4
-// TMA producer, warp 5 tcgen05 issuer.  TMEM: cross block [0, 256), self block [256, 384).
+// Roles: warps 0-7 epilogue (TMEM -> bf16 rows in the store's swizzled staging -> TMA stores), two
+// warps per TMEM lane quarter splitting the output columns, so one warp's TMEM loads and shared-memory
+// writes overlap the other's and the accumulator drains in about half the time; warp 8 TMA producer,
+// warp 9 tcgen05 issuer.  TMEM: cross block [0, 256), self block [256, 384).
 #include <type_traits>
 
 #include "lcb_sm100.h"
@@ -23,7 +25,8 @@
 namespace rocs {
 
 namespace {
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kStages = 2;
 constexpr int kMaxLd = 384;  // max output row length (n_r + n_c <= 256 + 128)
 
@@ -121,12 +124,12 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
     mbar_init(xr_full, 1);
     mbar_init(xr_empty, 1);
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, 8);
     mbar_init(drain_bar, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(s_tmem, 512);
     tmem_relinquish();
   }
@@ -135,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
 
-  if (ubeg < uend && warp == 4) {
+  if (ubeg < uend && warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_xr);
@@ -173,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
         if (n_xr > 0) mbar_drain(xr_full, (n_xr - 1) & 1, 20000000ull);
       }
     }
-  } else if (ubeg < uend && warp == 5) {
+  } else if (ubeg < uend && warp == kMmaWarp) {
     // ------------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
       const uint32_t id_cross = idesc_bf16(128, n_b, false, false);
@@ -215,9 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
       umma_commit(drain_bar);
       mbar_drain(drain_bar, 0, 50000000ull);
     }
-  } else if (ubeg < uend && warp < 4) {
-    // ------------------------------------------------------------------ epilogue warps 0..3
-    const int q = warp;
+  } else if (ubeg < uend && warp < 8) {
+    // ------------------------------------------------------------------ epilogue warps 0..7
+    // Two warps per TMEM lane quarter q share its 32 staging rows: warp q writes and stores the 64-column
+    // boxes below b_split = floor(n_r / 64) (whole cross-block boxes), warp q + 4 the boxes from b_split
+    // on (the rest of the cross block, the self block, the padding), so neither waits on the other.
+    const int q = warp & 3, half = warp >> 2;
+    const int b_split = n_r >> 6;
     const uint32_t t_lane = (uint32_t)(32 * q) << 16;
     uint8_t* stg = s_stg + q * L::kStgWarp;
     const uint32_t stg_u = smem_u32(stg);
@@ -282,18 +289,20 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
       if (!mbar_wait(acc_full, aph, ctl, 821)) break;
       tc_fence_after();
       if (valid) {
-        if (lane == 0) bulk_wait_read<0>();  // this warp's previous stores have read the staging rows
+        if (lane == 0) bulk_wait_read<0>();  // this warp's previous stores have read its staging boxes
         __syncwarp();
-        for (int uu = ncols >> 3; uu < nbox * 8; ++uu) st_shared_v4(unit_addr(uu), 0u, 0u, 0u, 0u);  // pad
+        if (half == 1)
+          for (int uu = ncols >> 3; uu < nbox * 8; ++uu) st_shared_v4(unit_addr(uu), 0u, 0u, 0u, 0u);  // pad
+        const int h_lo = half == 0 ? 0 : b_split, h_hi = half == 0 ? b_split : (n_r + 63) >> 6;
 #pragma unroll 1
-        for (int h = 0; 64 * h < n_r; ++h) {  // cross block (columns past n_r are the zero rows of B)
+        for (int h = h_lo; h < h_hi; ++h) {  // cross block (columns past n_r are the zero rows of B)
           uint32_t v[2][32];
           const int ch = n_r - 64 * h;
           load64(tmem_base + t_lane + 64 * h, v, ch > 32);
           put_aligned(64 * h, v[0], min(32, ch));
           if (ch > 32) put_aligned(64 * h + 32, v[1], min(32, ch - 32));
         }
-        if (cand) {  // self block: the n_c Gram columns of this row's own candidate
+        if (cand && half == 1) {  // self block: the n_c Gram columns of this row's own candidate
           const int cb = (32 * q / n_c) * n_c, sh = n_r & 7;
 #pragma unroll 1
           for (int h = 0; 64 * h < n_c; ++h) {
@@ -320,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          for (int b = 0; b < nbox; ++b) {
+          for (int b = half == 0 ? 0 : b_split; b < (half == 0 ? b_split : nbox); ++b) {
             if (cand) tma_store_2d(&p.tm_yc, stg + b * (32 * 128), b * 64, p.cand_off[r] * n_c + lrow0);
             else tma_store_3d(&p.tm_yr, stg + b * (32 * 128), b * 64, lrow0, r);
           }
@@ -334,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
