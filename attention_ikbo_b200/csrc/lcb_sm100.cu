@@ -33,7 +33,6 @@ namespace rocs {
 namespace {
 
 constexpr int kWarpsPerGroup = 4;  // one epilogue group covers the 128 TMEM lanes (tile rows)
-constexpr int kStages = 4;
 
 // NG epilogue groups of four warps, then the TMA producer warp and the tcgen05 issuer warp.
 // NG = 1: the group drains both TMEM accumulator buffers in turn; NG = 2: group g drains buffer g
@@ -51,7 +50,10 @@ constexpr int OC = 128;
 template <int D, int NC, int NG>
 struct LcbSmem {
   static constexpr int kEpiWarps = LcbRoles<NG>::kEpiWarps;
-  static constexpr int kStgPerWarp = 2 / NG;              // staging buffers per epilogue warp
+  // NG = 2 (block epilogue): two staging buffers per warp so the next tile's residual rows load while this
+  // tile is finished; the ring gives up two stages for them
+  static constexpr int kStages = NG == 2 ? 2 : 4;
+  static constexpr int kStgPerWarp = 2;                   // staging buffers per epilogue warp
   static constexpr uint32_t kWcc = NC * OC * 2;           // W_CC resident, NC/64 boxes of [128 x 64]
   static constexpr uint32_t kXc = NC * D * 2;             // one candidate's X^C tile
   static constexpr uint32_t kStgHalf = 32 * 128;          // 32 rows x 64 bf16 (one TMA store box)
@@ -91,8 +93,8 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
   float* s_gb = reinterpret_cast<float*>(smem + L::off_par);  // block epilogue: gamma_C [D], beta_C [D]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kStages;
-  uint64_t* acc_full = bars + 2 * kStages;
+  uint64_t* empty = bars + L::kStages;
+  uint64_t* acc_full = bars + 2 * L::kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* wq_full = acc_empty + 2;
   uint64_t* wq_empty = wq_full + 2;
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
   const int cbeg = (int)(((int64_t)C * b) / G), cend = (int)(((int64_t)C * (b + 1)) / G);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
           for (int cc = 0; cc < D / 64; ++cc)
             tma_load_2d(slot + 16384 + cc * 8192, &p.tm_xr, &full[s], cc * 64, r * p.n_r + kb * 64);
           ++n_issued;
-          if (++s == kStages) { s = 0; ph ^= 1; }
+          if (++s == L::kStages) { s = 0; ph ^= 1; }
         }
       }
       for (int i = cbeg; ok && i < cend; ++i) {  // candidate phase
@@ -188,11 +190,11 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
         mbar_arrive_expect_tx(&full[s], L::kXc);
         for (int cc = 0; cc < D / 64; ++cc) tma_load_2d(slot + cc * (NC * 128), &p.tm_xc, &full[s], cc * 64, i * NC);
         ++n_issued;
-        if (++s == kStages) { s = 0; ph ^= 1; }
+        if (++s == L::kStages) { s = 0; ph ^= 1; }
       }
       if (!ok) {  // let loads already in flight land before the CTA's shared memory goes away
-        for (int k = n_issued > kStages ? n_issued - kStages : 0; k < n_issued; ++k)
-          mbar_drain(&full[k % kStages], (k / kStages) & 1, 20000000ull);
+        for (int k = n_issued > L::kStages ? n_issued - L::kStages : 0; k < n_issued; ++k)
+          mbar_drain(&full[k % L::kStages], (k / L::kStages) & 1, 20000000ull);
         if (cbeg < cend) mbar_drain(wcc_bar, 0, 20000000ull);
       }
     }
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
           for (int kin = 0; kin < 4; ++kin)
             umma_ss(d_tmem, sdesc_add(ad, kin * 32), sdesc_add(bd, kin * 2048), idesc, (kb | kin) != 0);
           umma_commit(&empty[s]);
-          if (++s == kStages) { s = 0; ph ^= 1; }
+          if (++s == L::kStages) { s = 0; ph ^= 1; }
         }
         if (!ok) break;
         umma_commit(&acc_full[ab]);
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
           umma_ss(d_tmem, sdesc_add(wccd, (ks >> 2) * 16384 + (ks & 3) * 32), sdesc_add(bd, ks * 2048), idesc, ks != 0);
         umma_commit(&empty[s]);
         umma_commit(&acc_full[ab]);
-        if (++s == kStages) { s = 0; ph ^= 1; }
+        if (++s == L::kStages) { s = 0; ph ^= 1; }
         if (++ab == 2) { ab = 0; aph ^= 1; }
       }
       umma_commit(drain_bar);  // wait for every MMA this thread issued before TMEM is freed
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
         const int mid = (lo + hi + 1) >> 1;
         if (p.cand_off[mid] <= cbeg) lo = mid; else hi = mid - 1;
       }
-      int r = lo, next_off = p.cand_off[r + 1], r_staged = -1;
+      int r = lo, next_off = p.cand_off[r + 1], r_staged = -1, res_next = -1;
       for (int i = cbeg; i < cend; ++i) {
         while (i >= next_off) {
           if (++r >= R) break;
@@ -542,12 +544,12 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);
           store_tile(&p.tm_yc, stg_off, i * OC + 32 * quarter);
-        } else {  // candidate group's epilogue: residual prefetched before the accumulator is ready
+        } else {  // candidate group's epilogue: residual loaded one tile ahead into the other staging buffer
           const uint32_t stg_off = acquire_stage();
           const uint32_t stg = smem_u32(s_stg + stg_off);
           const bool res = p.epi_c.has_residual != 0;
           if (res) {
-            load_residual(&p.tm_res_c, stg_off, i * OC + 32 * quarter);
+            if (res_next != i) load_residual(&p.tm_res_c, stg_off, i * OC + 32 * quarter);
             // this group's tile after next: start its residual rows towards L2 now
             if (lane == 0 && i + 2 * NG < cend)
               for (int h = 0; h < D / 64; ++h) tma_prefetch_l2_2d(&p.tm_res_c, h * 64, (i + 2 * NG) * OC + 32 * quarter);
@@ -568,6 +570,14 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);
           store_tile(&p.tm_yc, stg_off, i * OC + 32 * quarter);
+          // this group's next tile: its residual rows into the other staging buffer (whose last store,
+          // two groups back, must have finished reading it)
+          if (res && i + NG < cend) {
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            load_residual(&p.tm_res_c, (uint32_t)((ew * L::kStgPerWarp + (sb ^ 1)) * L::kStgBuf), (i + NG) * OC + 32 * quarter);
+            res_next = i + NG;
+          }
         }
         next_stage();
         aphs ^= 1u << ab;
