@@ -20,7 +20,10 @@
 //     tile A, warps 8-11 of tile B.  S = Q K^T lands in TMEM (fp32), the softmax warps write
 //     P (bf16) back over S in TMEM, and P V is issued with P as the TMEM A operand, O
 //     accumulating in TMEM.  The issuer alternates [PV_A, S_A] and [PV_B, S_B] so the
-//     tensor core works on one tile while the softmax warps of the other tile run.
+//     tensor core works on one tile while the softmax warps of the other tile run.  With
+//     dh = 64 the O accumulators leave 128 TMEM columns free, so P gets columns of its own:
+//     the next S of a tile is issued as soon as the softmax has read the current one, and P
+//     is rewritten only after the previous P V has completed.
 //   * online softmax in the exp2 domain with lazy rescaling: O and the running sum are
 //     rescaled only when a row's maximum grows by more than 2^8; row maxima with 3-input max
 //     chains, exponent arguments and row sums with packed fp32x2 FMA/ADD, exp2 on the MUFU.
@@ -55,7 +58,7 @@ struct DcaSmem {
   static constexpr uint32_t off_q = 0;
   static constexpr uint32_t off_ring = 2 * kTile;
   static constexpr uint32_t off_bar = off_ring + kRing * kTile;
-  static constexpr uint32_t n_bars = 2 * kRing + 2 * 8 + 1;
+  static constexpr uint32_t n_bars = 2 * kRing + 2 * 8 + 1 + 4;
   static constexpr uint32_t off_misc = off_bar + n_bars * 8;
   static constexpr uint32_t bytes = off_misc + 64;
   static constexpr uint32_t alloc_bytes = bytes + 1024;
@@ -120,6 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
   uint64_t* wq_full = o_empty + 2;  // two-slot work queue: the producer runs one unit ahead
   uint64_t* wq_empty = wq_full + 2;
   uint64_t* drain_bar = wq_empty + 2;
+  uint64_t* s_free = drain_bar + 1;  // [2] separate-P layout: S of tile x read into registers
+  uint64_t* pv_done = s_free + 2;    // [2] separate-P layout: P V of tile x complete (P may be rewritten)
   int* s_wq = reinterpret_cast<int*>(smem + L::off_misc);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::off_misc + 16);
   int* s_abort = reinterpret_cast<int*>(smem + L::off_misc + 32);
@@ -140,6 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       mbar_init(&p_full[x], 4);
       mbar_init(&o_full[x], 1);
       mbar_init(&o_empty[x], 4);
+      mbar_init(&s_free[x], 4);
+      mbar_init(&pv_done[x], 1);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&wq_full[k], 1);
@@ -157,7 +164,11 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+DH) O_B [256+DH,256+2DH); P_X over S_X [0,64)
+  // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+DH) O_B [256+DH,256+2DH).  dh = 128: P_X over
+  // S_X [0,64), so S of the next K/V tile waits for P V.  dh = 64 leaves 128 columns free: P_A [384,448),
+  // P_B [448,512) of their own, so S of the next tile is computed while the softmax works on this one.
+  constexpr bool kSepP = 256 + 2 * DH + 128 <= 512;
+  constexpr uint32_t kPCol = 256 + 2 * DH;
 
   if (warp < kSoftmaxWarp0) {
    // warpgroup 0: hand registers to the softmax warpgroups, then producer / issuer / idle
@@ -246,10 +257,23 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       };
       auto issue_pv = [&](int x, uint32_t vslot, bool acc) {
         const uint64_t vd = sdesc_sw128(vslot, BN * 128, 1024);
+        const uint32_t pa = tmem_base + (kSepP ? kPCol + x * 64 : x * 128);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(tmem_base + 256 + x * DH, tmem_base + x * 128 + kk * 8, sdesc_add(vd, kk * 2048), idesc_o,
-                  (acc || kk != 0) ? 1u : 0u);
+          umma_ts(tmem_base + 256 + x * DH, pa + kk * 8, sdesc_add(vd, kk * 2048), idesc_o, (acc || kk != 0) ? 1u : 0u);
+      };
+      uint32_t sfph[2] = {0, 0};
+      bool s_pend[2] = {false, false};
+      // separate-P layout: S_x may be overwritten once the softmax has read the previous S_x
+      auto issue_s_free = [&](int x, uint32_t kslot) -> bool {
+        if (s_pend[x]) {
+          if (!mbar_wait(&s_free[x], sfph[x], ctl, 610)) return false;
+          sfph[x] ^= 1;
+          tc_fence_after();
+        }
+        issue_s(x, kslot);
+        s_pend[x] = true;
+        return true;
       };
       auto wait_p = [&](int x, bool first_pv) -> bool {
         if (!mbar_wait(&p_full[x], pph[x], ctl, 601)) return false;
@@ -280,6 +304,41 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         if (!next_slot(kslot, 605)) { ok = false; break; }
         advance();
         tc_fence_after();
+        if constexpr (kSepP) {
+          for (int x = 0; x < nx && ok; ++x) ok = issue_s_free(x, kslot);
+          if (!ok) break;
+          release_slot(kslot);
+          // per K/V step: S of the next tile as soon as the softmax has read the current one, then P V
+          for (int j = 1; j < w.nkv; ++j) {
+            if (!next_slot(kslot, 606)) { ok = false; break; }
+            advance();
+            for (int x = 0; x < nx && ok; ++x) ok = issue_s_free(x, kslot);
+            if (!ok) break;
+            release_slot(kslot);
+            if (!next_slot(vslot, 607)) { ok = false; break; }
+            advance();
+            for (int x = 0; x < nx; ++x) {
+              if (!wait_p(x, j == 1)) { ok = false; break; }
+              issue_pv(x, vslot, j > 1);
+              umma_commit(&pv_done[x]);
+            }
+            if (!ok) break;
+            release_slot(vslot);
+          }
+          if (!ok) break;
+          for (int x = 0; x < nx; ++x) umma_commit(&q_empty[x]);
+          if (!next_slot(vslot, 608)) { ok = false; break; }
+          advance();
+          for (int x = 0; x < nx; ++x) {
+            if (!wait_p(x, w.nkv == 1)) { ok = false; break; }
+            issue_pv(x, vslot, w.nkv > 1);
+            umma_commit(&pv_done[x]);
+            umma_commit(&o_full[x]);
+          }
+          if (!ok) break;
+          release_slot(vslot);
+          continue;
+        }
         issue_s(0, kslot);
         if (nx == 2) issue_s(1, kslot);
         release_slot(kslot);
@@ -320,9 +379,10 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
     const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
     const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
     const uint32_t s_addr = tmem_base + t_lane + x * 128;
+    const uint32_t p_addr = kSepP ? tmem_base + t_lane + kPCol + x * 64 : s_addr;
     const uint32_t o_addr = tmem_base + t_lane + 256 + x * DH;
     const float c = p.scale_log2;
-    uint32_t ws_ = 0, wph = 0, sph = 0, ofph = 0;
+    uint32_t ws_ = 0, wph = 0, sph = 0, ofph = 0, n_sig = 0;
     bool ok = true;
     for (;;) {
       if (!mbar_wait(&wq_full[ws_], wph, ctl, 701)) { ok = false; break; }
@@ -353,6 +413,17 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + c4 * 32, sv[c4]);
         tmem_ld_wait();
+        if constexpr (kSepP) {
+          // S is in registers: the next S may be computed; P is rewritten only once P V of the last
+          // handed-over P is complete (which also makes O current for a rescale)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[x]);
+          if (n_sig > 0) {
+            if (!mbar_wait(&pv_done[x], (n_sig - 1) & 1, ctl, 706)) { ok = false; break; }
+            tc_fence_after();
+          }
+        }
         const int kvalid = w.L - j * BN;
         if (kvalid < BN) {
 #pragma unroll
@@ -398,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
               else asm("add.f32x2 %0, %1, %2;" : "=l"(ls0) : "l"(ls0), "l"(ep));
               pk[k] = pack_bf16x2(p0, p1);
             }
-            tmem_st16(s_addr + c4 * 16, pk);
+            tmem_st16(p_addr + c4 * 16, pk);
           }
         };
         auto row_max = [&]() {
@@ -448,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[x]);
+        ++n_sig;
       }
       if (!ok) break;
       if (!mbar_wait(&o_full[x], ofph, ctl, 703)) { ok = false; break; }

@@ -115,3 +115,30 @@ def test_dca_long_full_size_sampled(ikbo, oracle_mod):
     x = ri.dca_long()
     o, lse = run_dca(ikbo, x)
     check(oracle_mod, x, o, lse, sel=_sample(x, 24, 3))
+
+
+def _f32_to_bf16(a):
+    """Round-to-nearest-even fp32 -> bf16 bits (finite inputs)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    return ((u + (((u >> 16) & 1) + 0x7FFF)) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("dh", [64, 128])
+def test_dca_growing_max_rescale(ikbo, oracle_mod, dh):
+    """Scores that grow along the key axis (non-negative queries and keys, keys scaled by a ramp): the row
+    maximum rises by far more than 2^8 (in exp2 units) from one 128-key tile to the next, so every tile
+    after the first takes the online softmax's rescale-and-redo path."""
+    x = ri.make_dca("t", [3, 40], [700, 300], 2, 2, dh, 31)
+    q = np.abs(ri.bf16_to_f32(x.q_t))
+    k = np.abs(ri.bf16_to_f32(x.k_t))
+    for r in range(len(x.seq_off) - 1):
+        s0, s1 = int(x.seq_off[r]), int(x.seq_off[r + 1])
+        k[s0:s1] *= (0.25 + 10.0 * np.arange(s1 - s0) / (s1 - s0))[:, None, None]
+    x.q_t, x.k_t = _f32_to_bf16(q), _f32_to_bf16(k)
+    # the premise: consecutive 128-key tiles' row maxima differ by more than 8 in log2 units
+    s = np.einsum("hd,khd->hk", ri.bf16_to_f32(x.q_t)[0].astype(np.float64),
+                  ri.bf16_to_f32(x.k_t)[:700].astype(np.float64)) * x.scale / np.log(2.0)
+    tile_max = np.array([s[:, t * 128:(t + 1) * 128].max() for t in range(5)])  # the five full tiles
+    assert np.all(np.diff(tile_max) > 8.0)
+    o, lse = run_dca(ikbo, x)
+    check(oracle_mod, x, o, lse)
