@@ -192,6 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         if (++rs == kRing) { rs = 0; rph ^= 1; }
         return true;
       };
+      // launched as a programmatic dependent of the scheduling kernel: the prologue above overlapped it;
+      // the unit table and the zeroed ticket are visible after this wait
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       while (ok) {
         const int t = atomicAdd(p.ticket, 1);
         const int item = t < p.n_units ? t : -1;
@@ -563,6 +566,8 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
 // Scratch (workspace): len[R], sorted[R], start[R+1].
 // ------------------------------------------------------------------------------------
 __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
+  // the attention kernel may start its prologue now; it waits for this grid before claiming units
+  asm volatile("griddepcontrol.launch_dependents;");
   int* len = p.scratch;
   int* sorted = len + p.R;
   int* start = sorted + p.R;
@@ -637,8 +642,19 @@ static cudaError_t launch_t(const DcaParams& p, int grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k<<<grid, kThreads, L::alloc_bytes, st>>>(p);
-  return cudaGetLastError();
+  // programmatic dependent launch: set-up (barriers, TMEM, descriptor prefetch) overlaps the scheduling
+  // kernel that precedes it on the stream
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::alloc_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, p);
 }
 
 cudaError_t launch_dca_sm100(const DcaParams& p, int dh, int grid, cudaStream_t st) {
