@@ -1,0 +1,111 @@
+"""Seeded random configurations of the LCB, DCA and FM against the fp64 oracle.
+
+Shapes, CSR offsets (empty requests and candidate-free requests included), key lengths and token counts are
+drawn from a fixed generator; each case checks every request output and a sample of candidate outputs
+(the sampled rows include the first and last candidate, where tiles and requests begin and end).
+Operations: ROCS (arXiv:2607.27744) section 3.1.2 Eq. (6) / section 4.1 Eq. (14) for the LCB, section 3.2
+Eq. (13) for the DCA, section 3.1.4 Eq. (10) for the FM.
+"""
+import numpy as np
+import pytest
+import torch
+
+import rocs_inputs as ri
+from _helpers import assert_close, dev, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ikbo():
+    import attention_ikbo_b200 as m
+
+    m.load_library()
+    return m
+
+
+def _status_ok(ikbo, ws):
+    code, detail = ikbo.rocs_read_status(ws)
+    assert code == 0, f"device status {ikbo.STATUS_NAMES.get(code)} at {detail}"
+
+
+def _sample(rng, C, n):
+    if C <= n:
+        return np.arange(C)
+    return np.unique(np.concatenate([[0, C - 1], rng.choice(C, n - 2, replace=False)]))
+
+
+def _counts(rng, R, hi):
+    c = rng.integers(0, hi + 1, R)
+    c[rng.random(R) < 0.2] = 0
+    return c
+
+
+LCB_CASES = list(range(24))
+
+
+@pytest.mark.parametrize("case", LCB_CASES)
+def test_lcb_random(ikbo, oracle_mod, case):
+    rng = np.random.default_rng(1000 + case)
+    R = int(rng.integers(1, 6))
+    n_r = int(rng.choice([64, 128, 192, 256]))
+    n_c, d, o_r = int(rng.choice([64, 128])), int(rng.choice([64, 128])), int(rng.choice([128, 256]))
+    x = ri.make_lcb("fuzz", _counts(rng, R, 40), n_r, n_c, d, o_r, 128, 50 + case, "bf16")
+    args = [dev(a) for a in (x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)]
+    y_req, y_cand = ikbo.rocs_lcb_forward(*args, x.cand_off)
+    _status_ok(ikbo, ikbo.rocs_lcb_forward.last_workspace)
+    sel = _sample(rng, x.C, 24)
+    yr, yc = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, sel_req=np.arange(x.R), sel_cand=sel)
+    assert_close(host_f64(y_req), yr, "bf16", "Y^R")
+    if len(sel):
+        assert_close(host_f64(y_cand[torch.as_tensor(sel, device=y_cand.device)]), yc, "bf16", "Y^C")
+
+
+DCA_CASES = list(range(32))
+
+
+@pytest.mark.parametrize("case", DCA_CASES)
+def test_dca_random(ikbo, oracle_mod, case):
+    rng = np.random.default_rng(2000 + case)
+    R = int(rng.integers(1, 6))
+    counts = _counts(rng, R, 300)
+    lengths = rng.integers(0, 900, R)
+    lengths[rng.random(R) < 0.15] = 0
+    q, H, dh = int(rng.choice([1, 2, 3, 4])), int(rng.choice([1, 2, 4])), int(rng.choice([64, 128]))
+    x = ri.make_dca("fuzz", counts, lengths, q, H, dh, 70 + case)
+    o, lse = ikbo.rocs_dca_forward(dev(x.q_t), dev(x.k_t), dev(x.v_t), x.cand_off, x.seq_off, x.q, x.scale)
+    _status_ok(ikbo, ikbo.rocs_dca_forward.last_workspace)
+    sel = _sample(rng, x.C, 32)
+    if not len(sel):
+        return
+    oo, ll = oracle_mod.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, x.v_t, x.q, x.scale, sel_cand=sel)
+    rows = torch.as_tensor((sel[:, None] * x.q + np.arange(x.q)[None, :]).ravel(), device=o.device)
+    assert_close(host_f64(o[rows]).reshape(oo.shape), oo, "bf16", "O")
+    got_l = host_f64(lse[rows]).reshape(ll.shape)
+    fin = np.isfinite(ll)
+    assert np.array_equal(np.isfinite(got_l), fin) and np.all(got_l[~fin] == -np.inf)
+    if fin.any():
+        assert_close(got_l[fin], ll[fin], "bf16", "LSE")
+
+
+FM_CASES = list(range(24))
+
+
+@pytest.mark.parametrize("case", FM_CASES)
+def test_fm_random(ikbo, oracle_mod, case):
+    rng = np.random.default_rng(3000 + case)
+    R = int(rng.integers(1, 6))
+    n_r = 2 * int(rng.integers(1, 129))
+    n_c, d = int(rng.choice([32, 64, 128])), int(rng.choice([64, 128]))
+    x = ri.make_fm("fuzz", _counts(rng, R, 50), n_r, n_c, d, 90 + case)
+    y_req, y_cand = ikbo.rocs_fm_forward(dev(x.x_req), dev(x.x_cand), x.cand_off)
+    _status_ok(ikbo, ikbo.rocs_fm_forward.last_workspace)
+    sel = _sample(rng, x.C, 32)
+    yr, yc = oracle_mod.fm(x.cand_off, x.x_req, x.x_cand, sel_cand=sel)
+    gr = host_f64(y_req)
+    assert_close(gr[:, :, :n_r], yr, "bf16", "Y^R")
+    assert not np.any(gr[:, :, n_r:])
+    if len(sel):
+        gc = host_f64(y_cand[torch.as_tensor(sel, device=y_cand.device)])
+        assert_close(gc[:, :, :n_r + n_c], yc, "bf16", "Y^C")
+        assert not np.any(gc[:, :, n_r + n_c:])
