@@ -109,3 +109,37 @@ def test_fm_random(ikbo, oracle_mod, case):
         gc = host_f64(y_cand[torch.as_tensor(sel, device=y_cand.device)])
         assert_close(gc[:, :, :n_r + n_c], yc, "bf16", "Y^C")
         assert not np.any(gc[:, :, n_r + n_c:])
+
+
+BLOCK_CASES = list(range(16))
+
+
+def _epi_dev(e):
+    out = {"eps": e.eps, "norm": e.norm, "act": e.act}
+    for k in ("bias", "gamma", "beta", "residual"):
+        v = getattr(e, k)
+        if v is not None:
+            out[k] = dev(v)
+    return out
+
+
+@pytest.mark.parametrize("case", BLOCK_CASES)
+def test_lcb_block_random(ikbo, oracle_mod, case):
+    """LCB block (section 3.1.3 Eq. (7)-(8) epilogues): each group's norm and activation drawn independently."""
+    rng = np.random.default_rng(4000 + case)
+    R = int(rng.integers(1, 5))
+    n_r = int(rng.choice([64, 128, 256]))
+    n_c, d, o_r = int(rng.choice([64, 128])), int(rng.choice([64, 128])), int(rng.choice([128, 256]))
+    norms, acts = ["none", "layernorm", "rmsnorm"], ["none", "relu", "silu", "gelu"]
+    x = ri.make_lcb_block("fuzz", _counts(rng, R, 30), n_r, n_c, d, o_r, 128, 110 + case,
+                          str(rng.choice(norms)), str(rng.choice(acts)), residual=bool(rng.random() < 0.6),
+                          norm_r=str(rng.choice(norms)), act_r=str(rng.choice(acts)))
+    L = x.lcb
+    args = [dev(a) for a in (L.x_req, L.x_cand, L.w_rr, L.w_cr, L.w_cc)]
+    y_req, y_cand = ikbo.rocs_lcb_block_forward(*args, L.cand_off, _epi_dev(x.epi_r), _epi_dev(x.epi_c))
+    _status_ok(ikbo, ikbo.rocs_lcb_block_forward.last_workspace)
+    sel = _sample(rng, L.C, 24)
+    yr, yc = oracle_mod.lcb_block(L.cand_off, L.x_req, L.x_cand, L.w_rr, L.w_cr, L.w_cc, x.epi_r, x.epi_c, sel_cand=sel)
+    assert_close(host_f64(y_req), yr, "bf16", "Y^R")
+    if len(sel):
+        assert_close(host_f64(y_cand[torch.as_tensor(sel, device=y_cand.device)]), yc, "bf16", "Y^C")
