@@ -685,7 +685,9 @@ def ncu_traffic(p):
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        d = json.load(f).get(p.name)
+        table = json.load(f)
+    # entries are keyed by part name, or "name@inputs" where one part name is captured on several inputs
+    d = table.get(f"{p.name}@{part_signature(p)}") or table.get(p.name)
     if not d or d.get("src_sha") != kernel_sha(p.kernel) or d.get("inputs") != part_signature(p):
         return None
     return d["dram_bytes_per_unit"] * p.units
