@@ -143,3 +143,39 @@ def test_lcb_block_random(ikbo, oracle_mod, case):
     assert_close(host_f64(y_req), yr, "bf16", "Y^R")
     if len(sel):
         assert_close(host_f64(y_cand[torch.as_tensor(sel, device=y_cand.device)]), yc, "bf16", "Y^C")
+
+
+def test_many_small_requests(ikbo, oracle_mod):
+    """3,000 requests of 0-3 candidates (more requests than the scheduling kernels' 1,024 threads): the LCB,
+    FM and DCA tile tables and request lookups across thread partitions, checked on sampled candidates."""
+    rng = np.random.default_rng(5000)
+    counts = rng.integers(0, 4, 3000)
+    x = ri.make_lcb("many", counts, 64, 64, 64, 128, 128, 131, "bf16")
+    args = [dev(a) for a in (x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)]
+    y_req, y_cand = ikbo.rocs_lcb_forward(*args, x.cand_off)
+    _status_ok(ikbo, ikbo.rocs_lcb_forward.last_workspace)
+    sel = _sample(rng, x.C, 48)
+    sel_req = np.unique(np.concatenate([[0, x.R - 1], rng.choice(x.R, 30, replace=False)]))
+    yr, yc = oracle_mod.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, sel_req=sel_req, sel_cand=sel)
+    assert_close(host_f64(y_req[torch.as_tensor(sel_req, device=y_req.device)]), yr, "bf16", "Y^R")
+    assert_close(host_f64(y_cand[torch.as_tensor(sel, device=y_cand.device)]), yc, "bf16", "Y^C")
+
+    f = ri.make_fm("many", counts, 34, 32, 64, 132)
+    fr, fc = ikbo.rocs_fm_forward(dev(f.x_req), dev(f.x_cand), f.cand_off)
+    _status_ok(ikbo, ikbo.rocs_fm_forward.last_workspace)
+    yr, yc = oracle_mod.fm(f.cand_off, f.x_req, f.x_cand, sel_cand=sel)
+    assert_close(host_f64(fr)[:, :, :34], yr, "bf16", "FM Y^R")
+    assert_close(host_f64(fc[torch.as_tensor(sel, device=fc.device)])[:, :, :66], yc, "bf16", "FM Y^C")
+
+    lengths = rng.integers(0, 200, 3000)
+    d = ri.make_dca("many", counts, lengths, 2, 2, 64, 133)
+    o, lse = ikbo.rocs_dca_forward(dev(d.q_t), dev(d.k_t), dev(d.v_t), d.cand_off, d.seq_off, d.q, d.scale)
+    _status_ok(ikbo, ikbo.rocs_dca_forward.last_workspace)
+    oo, ll = oracle_mod.dca(d.cand_off, d.seq_off, d.q_t, d.k_t, d.v_t, d.q, d.scale, sel_cand=sel)
+    rows = torch.as_tensor((sel[:, None] * d.q + np.arange(d.q)[None, :]).ravel(), device=o.device)
+    assert_close(host_f64(o[rows]).reshape(oo.shape), oo, "bf16", "DCA O")
+    got_l = host_f64(lse[rows]).reshape(ll.shape)
+    fin = np.isfinite(ll)
+    assert np.array_equal(np.isfinite(got_l), fin)
+    if fin.any():
+        assert_close(got_l[fin], ll[fin], "bf16", "DCA LSE")
