@@ -179,3 +179,22 @@ def test_many_small_requests(ikbo, oracle_mod):
     assert np.array_equal(np.isfinite(got_l), fin)
     if fin.any():
         assert_close(got_l[fin], ll[fin], "bf16", "DCA LSE")
+
+
+def test_dca_very_many_requests(ikbo, oracle_mod):
+    """More requests than the scheduling kernel ranks by key length (9,000): the unit table keeps request
+    order; sampled candidates against the oracle."""
+    rng = np.random.default_rng(5001)
+    counts, lengths = rng.integers(0, 3, 9000), rng.integers(0, 160, 9000)
+    d = ri.make_dca("vmany", counts, lengths, 1, 1, 128, 134)
+    o, lse = ikbo.rocs_dca_forward(dev(d.q_t), dev(d.k_t), dev(d.v_t), d.cand_off, d.seq_off, d.q, d.scale)
+    _status_ok(ikbo, ikbo.rocs_dca_forward.last_workspace)
+    sel = _sample(rng, d.C, 48)
+    oo, ll = oracle_mod.dca(d.cand_off, d.seq_off, d.q_t, d.k_t, d.v_t, d.q, d.scale, sel_cand=sel)
+    rows = torch.as_tensor(sel, device=o.device)
+    assert_close(host_f64(o[rows]).reshape(oo.shape), oo, "bf16", "O")
+    got_l = host_f64(lse[rows]).reshape(ll.shape)
+    fin = np.isfinite(ll)
+    assert np.array_equal(np.isfinite(got_l), fin)
+    if fin.any():
+        assert_close(got_l[fin], ll[fin], "bf16", "LSE")
