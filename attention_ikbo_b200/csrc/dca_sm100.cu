@@ -76,6 +76,22 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
+// tcgen05.wait::ld that also names 64 registers of the second half of S as in/out operands, so the compiler
+// keeps every use of them after the wait
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&a)[32], uint32_t (&b)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+                 "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]),
+                 "+r"(a[16]), "+r"(a[17]), "+r"(a[18]), "+r"(a[19]), "+r"(a[20]), "+r"(a[21]), "+r"(a[22]), "+r"(a[23]),
+                 "+r"(a[24]), "+r"(a[25]), "+r"(a[26]), "+r"(a[27]), "+r"(a[28]), "+r"(a[29]), "+r"(a[30]), "+r"(a[31]),
+                 "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]),
+                 "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15]),
+                 "+r"(b[16]), "+r"(b[17]), "+r"(b[18]), "+r"(b[19]), "+r"(b[20]), "+r"(b[21]), "+r"(b[22]), "+r"(b[23]),
+                 "+r"(b[24]), "+r"(b[25]), "+r"(b[26]), "+r"(b[27]), "+r"(b[28]), "+r"(b[29]), "+r"(b[30]), "+r"(b[31])
+               :
+               : "memory");
+}
+
 struct Unit {
   int r, h, row0;  // request, head, first query row (within the request's rows)
   int rows;        // query rows of the request (q * N_r)
@@ -413,9 +429,15 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         sph ^= 1;
         tc_fence_after();
         uint32_t sv[4][32];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_addr + c4 * 32, sv[c4]);
+        // first half of S, then the second half in flight while the first half's exponentials run (steady
+        // state of a full tile); the first tile of a unit and partial tiles wait for all of it
+        const bool split_ld = !kSepP && j > 0 && w.L - j * BN >= BN;
+        tmem_ld32(s_addr, sv[0]);
+        tmem_ld32(s_addr + 32, sv[1]);
         tmem_ld_wait();
+        tmem_ld32(s_addr + 64, sv[2]);
+        tmem_ld32(s_addr + 96, sv[3]);
+        if (!split_ld) tmem_ld_wait_regs(sv[2], sv[3]);
         if constexpr (kSepP) {
           // S is in registers: the next S may be computed; P is rewritten only once P V of the last
           // handed-over P is complete (which also makes O current for a rescale)
@@ -452,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
           for (int k = 0; k < 8; ++k) mq[k] = -INFINITY;
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
+            if (c4 == 2 && split_ld && with_max) tmem_ld_wait_regs(sv[2], sv[3]);
             uint32_t pk[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
