@@ -161,6 +161,9 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
         for (int kc = 0; kc < NC / 64; ++kc) tma_load_2d(s_wcc + kc * 16384, &p.tm_wcc, wcc_bar, kc * 64, 0);
       }
       uint32_t s = 0, ph = 0, qs = 0, qph = 0;
+      // launched as a programmatic dependent of the kernel that zeroes the ticket and the ready flags: the
+      // set-up above overlapped it; they are zero and visible to the whole grid after this wait
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       while (ok) {  // request phase: claim tiles until the ticket runs past the last request tile
         const int t = atomicAdd(&p.ws->counter, 1);
         const int item = t < n_req_tiles ? t : -1;
@@ -608,7 +611,32 @@ static cudaError_t launch_t(const LcbParams& p, int grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k<<<grid, LcbRoles<NG>::kThreads, L::alloc_bytes, st>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(LcbRoles<NG>::kThreads);
+  cfg.dynamicSmemBytes = L::alloc_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, p);
+}
+
+__global__ void rocs_zero_ints_kernel(int* a, int na, int* b, int nb) {
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int t = blockIdx.x * blockDim.x + threadIdx.x, n = gridDim.x * blockDim.x;
+  for (int i = t; i < na; i += n) a[i] = 0;
+  for (int i = t; i < nb; i += n) b[i] = 0;
+}
+
+cudaError_t launch_zero_ints(int* a, int na, int* b, int nb, cudaStream_t st) {
+  const int n = na > nb ? na : nb;
+  int grid = (n + 255) / 256;
+  if (grid > 64) grid = 64;
+  if (grid < 1) grid = 1;
+  rocs_zero_ints_kernel<<<grid, 256, 0, st>>>(a, na, b, nb);
   return cudaGetLastError();
 }
 

@@ -25,6 +25,9 @@ struct LcbParams {
   CUtensorMap tm_res_c;     // residual of Y^C viewed as [C*o_c, d], box {64, 32} (loads)
   EpiGroup epi_r, epi_c;
 };
+// Zeroes a[0:na] and b[0:nb] (the workspace header and the request ready flags) and lets the LCB kernel that
+// follows on the stream start its set-up before it finishes (programmatic dependent launch).
+cudaError_t launch_zero_ints(int* a, int na, int* b, int nb, cudaStream_t st);
 cudaError_t launch_lcb_sm100(const LcbParams& p, int d, int n_c, bool epilogue, int grid, cudaStream_t st);
 
 // fp32 CUDA-core IKBO-LCB (two launches: request GEMM, then candidate GEMM + fused Z add).

@@ -187,12 +187,10 @@ EpiGroup epi_group(const rocs_lcb_epilogue* e) {
 int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaStream_t st, int* launches,
             const LcbOpts& opts = LcbOpts()) {
   const LcbLayout L = lcb_body(a->R, a->o_c, a->d);
-  if (w == reinterpret_cast<uint8_t*>(hdr + 1)) {
-    if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader) + (size_t)a->R * sizeof(int), st) != cudaSuccess) return ROCS_ERR_CUDA;
-  } else if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess ||
-             cudaMemsetAsync(w, 0, (size_t)a->R * sizeof(int), st) != cudaSuccess) {
+  static_assert(sizeof(WsHeader) % sizeof(int) == 0, "header zeroed as ints");
+  if (launch_zero_ints(reinterpret_cast<int*>(hdr), (int)(sizeof(WsHeader) / sizeof(int)), reinterpret_cast<int*>(w + L.flags),
+                       (int)a->R, st) != cudaSuccess)
     return ROCS_ERR_CUDA;
-  }
   if (a->R == 0) return ROCS_OK;
   if (a->dtype == ROCS_F32) {
     LcbF32Params p;
