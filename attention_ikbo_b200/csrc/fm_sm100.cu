@@ -68,6 +68,8 @@ __device__ __forceinline__ void unit_walk_advance(UnitWalk& w, const int32_t* un
 
 // unit_off[r] = sum over requests s < r of (req_tiles + ceil(N_s * n_c / 128)); unit_off[R] = total
 __global__ void rocs_fm_schedule_kernel(const int32_t* cand_off, int32_t* unit_off, int R, int n_c, int req_tiles) {
+  // the FM kernel may start its set-up now; it waits for this grid before reading the unit offsets
+  asm volatile("griddepcontrol.launch_dependents;");
   __shared__ int s_part[1024];
   const int T = blockDim.x, t = threadIdx.x;
   const int per = (R + T - 1) / T;
@@ -137,6 +139,9 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_fm_sm100_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  // launched as a programmatic dependent of the scheduling kernel: the set-up above overlapped it; every
+  // role reads the unit offsets it wrote, so every thread waits for it here
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (ubeg < uend && warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
@@ -365,8 +370,17 @@ static cudaError_t launch_t(const FmParams& p, int grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k<<<grid, kThreads, L::alloc_bytes, st>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::alloc_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, p);
 }
 
 cudaError_t launch_fm_sm100(const FmParams& p, int d, int grid, cudaStream_t st) {
