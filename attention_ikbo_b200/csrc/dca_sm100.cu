@@ -667,17 +667,7 @@ static cudaError_t launch_t(const DcaParams& p, int grid, cudaStream_t st) {
   }
   // programmatic dependent launch: set-up (barriers, TMEM, descriptor prefetch) overlaps the scheduling
   // kernel that precedes it on the stream
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = L::alloc_bytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k, p);
+  return launch_dependent(k, grid, kThreads, L::alloc_bytes, st, p);
 }
 
 cudaError_t launch_dca_sm100(const DcaParams& p, int dh, int grid, cudaStream_t st) {

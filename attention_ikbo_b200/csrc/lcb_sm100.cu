@@ -611,17 +611,7 @@ static cudaError_t launch_t(const LcbParams& p, int grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(LcbRoles<NG>::kThreads);
-  cfg.dynamicSmemBytes = L::alloc_bytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k, p);
+  return launch_dependent(k, grid, LcbRoles<NG>::kThreads, L::alloc_bytes, st, p);
 }
 
 __global__ void rocs_zero_ints_kernel(int* a, int na, int* b, int nb) {
