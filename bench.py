@@ -42,6 +42,10 @@ KERNEL_SRC = {"lcb": "attention_ikbo_b200/csrc/lcb_sm100.cu", "dca": "attention_
               "fm": "attention_ikbo_b200/csrc/fm_sm100.cu"}
 
 
+# threads of every oracle call the bench makes (0: all host cores)
+ORACLE_THREADS = 0
+
+
 # ----------------------------------------------------------------------------------- parts
 class Part:
     name = ""
@@ -121,7 +125,8 @@ class LcbPart(Part):
         rs = np.random.RandomState(seed)
         sel = rs.choice(x.C, size=min(n, x.C), replace=False)
         t0 = time.perf_counter()
-        oracle.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, sel_req=[], sel_cand=sel)
+        oracle.lcb(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, sel_req=[], sel_cand=sel,
+                   nthreads=ORACLE_THREADS)
         return time.perf_counter() - t0, len(sel) / x.C
 
 
@@ -190,7 +195,7 @@ class LcbBlockPart(LcbPart):
         sel = rs.choice(x.C, size=min(n, x.C), replace=False)
         t0 = time.perf_counter()
         oracle.lcb_block(x.cand_off, x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc, b.epi_r, b.epi_c, sel_req=[],
-                         sel_cand=sel)
+                         sel_cand=sel, nthreads=ORACLE_THREADS)
         return time.perf_counter() - t0, len(sel) / x.C
 
 
@@ -262,7 +267,7 @@ class FmPart(Part):
         rs = np.random.RandomState(seed)
         sel = rs.choice(x.C, size=min(n, x.C), replace=False)
         t0 = time.perf_counter()
-        oracle.fm(x.cand_off, x.x_req, x.x_cand, sel_req=[], sel_cand=sel)
+        oracle.fm(x.cand_off, x.x_req, x.x_cand, sel_req=[], sel_cand=sel, nthreads=ORACLE_THREADS)
         return time.perf_counter() - t0, len(sel) / x.C
 
 
@@ -352,7 +357,7 @@ class DcaPart(Part):
         m = np.repeat(np.arange(x.R), np.diff(x.cand_off))
         frac = float(L[m[sel]].sum()) / float(L[m].sum())
         t0 = time.perf_counter()
-        oracle.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, x.v_t, x.q, x.scale, sel_cand=sel)
+        oracle.dca(x.cand_off, x.seq_off, x.q_t, x.k_t, x.v_t, x.q, x.scale, sel_cand=sel, nthreads=ORACLE_THREADS)
         return time.perf_counter() - t0, frac
 
 
@@ -443,7 +448,7 @@ class DcaBlockPart(Part):
         frac = float(L[m[sel]].sum()) / float(L[m].sum())
         t0 = time.perf_counter()
         oracle.dca_block(b.cand_off, b.seq_off, b.s_seq, *b.weights(), b.q_c, b.q_r, b.q, b.q_req, b.scale,
-                         sel_cand=sel, sel_req=[])
+                         sel_cand=sel, sel_req=[], nthreads=ORACLE_THREADS)
         return time.perf_counter() - t0, frac
 
 
@@ -488,7 +493,7 @@ class ProjPart(Part):
         sel = rs.choice(self.M, size=min(n, self.M), replace=False)
         y = ri.normal(seed, 99, (len(sel), self.K))  # the projection's cost does not depend on the values
         t0 = time.perf_counter()
-        oracle.proj(y, ci.w_q)
+        oracle.proj(y, ci.w_q, nthreads=ORACLE_THREADS)
         return time.perf_counter() - t0, len(sel) / self.M
 
 
@@ -578,7 +583,7 @@ class ChainOracle:
         w_dca = 4 * ci.H * ci.dh * L[m]
         frac = float((w_fixed + w_dca[sel]).sum()) / float((w_fixed + w_dca).sum())
         t0 = time.perf_counter()
-        oracle.chain(ci, sel, round_y=self.round_y)
+        oracle.chain(ci, sel, nthreads=ORACLE_THREADS, round_y=self.round_y)
         return time.perf_counter() - t0, frac
 
 
@@ -740,20 +745,31 @@ def reduce_max(x: float, dist, device) -> float:
 
 
 # ----------------------------------------------------------------------------------- arms
-def cpu_baseline(parts, oracle, budget_s=12.0):
-    """fp64 oracle on a bounded random sample of each part, scaled to the full step."""
+def cpu_baseline(parts, oracle, budget_s=12.0, single_budget_s=3.0):
+    """fp64 oracle on a bounded random sample of each part, scaled to the full step: on all host cores, and
+    (a smaller sample) on one core, extrapolated the same way."""
+    global ORACLE_THREADS
     est = 0.0
     desc = []
     for i, p in enumerate(parts):
         t1, f1 = p.oracle_sample(oracle, 2, 100 + i)  # calibration
-        per = max(t1 / max(f1, 1e-12), 1e-9)  # seconds for the whole part
         unit_time = t1 / 2
         n = int(max(2, min(4096, (budget_s / len(parts)) / max(unit_time, 1e-6))))
         t, f = p.oracle_sample(oracle, n, 200 + i)
         est += t / f
         desc.append(f"{p.name}: {n} random candidates ({100 * f:.3f}% of the part) in {t:.1f} s")
-        del per
-    return est, "; ".join(desc)
+    est1, desc1 = 0.0, []
+    ORACLE_THREADS = 1
+    try:
+        for i, p in enumerate(parts):
+            t1, f1 = p.oracle_sample(oracle, 1, 300 + i)  # calibration
+            n = int(max(1, min(4096, (single_budget_s / len(parts)) / max(t1, 1e-6))))
+            t, f = p.oracle_sample(oracle, n, 400 + i)
+            est1 += t / f
+            desc1.append(f"{p.name}: {n} random candidates ({100 * f:.3f}% of the part) in {t:.1f} s")
+    finally:
+        ORACLE_THREADS = 0
+    return est, "; ".join(desc), est1, "; ".join(desc1)
 
 
 def run_reference(args):
@@ -948,9 +964,12 @@ def run_ikbo(args):
         import oracle
 
         oracle.build_lib()
-        est_s, sample = cpu_baseline(oracle_parts(args.workload, parts), oracle, args.cpu_budget)
+        est_s, sample, est1, sample1 = cpu_baseline(oracle_parts(args.workload, parts), oracle, args.cpu_budget)
         cpu = {"value": step_flops / est_s / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
-               "sample": sample, "est_seconds_per_step": est_s}
+               "sample": sample, "est_seconds_per_step": est_s,
+               "single_thread": {"value": step_flops / est1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                                 "sample": sample1 + " (extrapolated to the whole step)",
+                                 "est_seconds_per_step": est1}}
 
     cfg = workload_config(args.workload, parts)
     cfg.update({"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
