@@ -83,9 +83,22 @@ std::vector<int64_t> index_map(const int32_t* off, int64_t R) {
   return m;
 }
 
+// the process default thread count (all host cores unless OMP_NUM_THREADS says otherwise), taken before
+// any call changes it
+int default_threads() {
+#ifdef _OPENMP
+  static const int n = omp_get_max_threads();
+  return n;
+#else
+  return 1;
+#endif
+}
+
+// nthreads > 0: that many OpenMP threads for this call; 0: the process default, also after an earlier call
+// asked for fewer
 void set_threads(int nthreads) {
 #ifdef _OPENMP
-  if (nthreads > 0) omp_set_num_threads(nthreads);
+  omp_set_num_threads(nthreads > 0 ? nthreads : default_threads());
 #else
   (void)nthreads;
 #endif
@@ -272,13 +285,7 @@ void lcb_block_request(const LcbDims& D, const void* x_req, const std::vector<do
 
 extern "C" {
 
-int rocs_oracle_max_threads(void) {
-#ifdef _OPENMP
-  return omp_get_max_threads();
-#else
-  return 1;
-#endif
-}
+int rocs_oracle_max_threads(void) { return default_threads(); }
 
 // IKBO-LCB oracle.  dtype 0 = fp32 inputs, 1 = bf16 inputs (bit patterns).
 // Computes Y^R for the requests listed in sel_req (y_req: [n_sel_req, o_r, d]) and
