@@ -95,7 +95,7 @@ class LcbPart(Part):
         return ikbo.last_launch_count()
 
     # -- host-resident batch through rocs_lcb_forward_host (copies pipelined with compute)
-    host_chunks = 16
+    host_chunks = 8
 
     def host_run(self, ikbo):
         """One step from pinned host inputs to pinned host outputs; returns (h2d bytes, d2h bytes)."""
@@ -317,7 +317,7 @@ class DcaPart(Part):
         return ikbo.last_launch_count()
 
     # -- host-resident batch through rocs_dca_forward_host (only when Q comes from the host)
-    host_chunks = 4
+    host_chunks = 2
 
     def host_run(self, ikbo):
         if len(self.h_in) != 3:
