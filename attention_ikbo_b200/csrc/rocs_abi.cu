@@ -191,6 +191,7 @@ int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaSt
   if (launch_zero_ints(reinterpret_cast<int*>(hdr), (int)(sizeof(WsHeader) / sizeof(int)), reinterpret_cast<int*>(w + L.flags),
                        (int)a->R, st) != cudaSuccess)
     return ROCS_ERR_CUDA;
+  *launches = 1;  // the zeroing kernel
   if (a->R == 0) return ROCS_OK;
   if (a->dtype == ROCS_F32) {
     LcbF32Params p;
@@ -212,7 +213,7 @@ int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaSt
     p.o_r = (int)a->o_r;
     p.o_c = (int)a->o_c;
     if (launch_lcb_f32(p, st) != cudaSuccess) return ROCS_ERR_CUDA;
-    *launches = C > 0 ? 2 : 1;
+    *launches = 1 + (C > 0 ? 2 : 1);
     return ROCS_OK;
   }
   LcbParams p;
@@ -255,7 +256,7 @@ int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaSt
   if (grid > sm_count()) grid = sm_count();
   if (grid < 1) grid = 1;
   if (launch_lcb_sm100(p, (int)a->d, (int)a->n_c, opts.block, (int)grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
-  *launches = 1;
+  *launches = 2;  // zeroing kernel + LCB kernel
   return ROCS_OK;
 }
 

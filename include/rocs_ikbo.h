@@ -109,7 +109,8 @@ typedef struct {
 /* Bytes of workspace rocs_lcb_forward needs for these sizes (0 if the sizes are invalid). */
 ROCS_API size_t rocs_lcb_workspace_size(const rocs_lcb_args* args);
 
-/* IKBO-LCB forward.  One kernel launch (bf16) or two (fp32) plus one memset, on `stream`. */
+/* IKBO-LCB forward, on `stream`: a kernel that zeroes the workspace header and the ready flags, then the
+ * LCB kernel (bf16, launched as its programmatic dependent) or the two fp32 kernels. */
 ROCS_API int rocs_lcb_forward(const rocs_lcb_args* args, rocs_stream_t stream);
 
 /* Explicit-expand baseline (ablation, not the method): materialises X^R per candidate
@@ -173,7 +174,7 @@ ROCS_API int rocs_lcb_forward_noalloc(const rocs_lcb_args* args, rocs_stream_t s
  *   norm     ROCS_NORM_*;  act ROCS_ACT_*;  eps >= 0 and finite
  * dtype must be ROCS_BF16 (else ROCS_ERR_UNSUPPORTED); sizes, workspace and errors as for
  * rocs_lcb_forward (workspace: rocs_lcb_workspace_size).  A NULL epilogue pointer means no
- * epilogue for that group.  One kernel launch plus one memset.
+ * epilogue for that group.  Two kernel launches (the zeroing kernel and the LCB kernel).
  * ---------------------------------------------------------------------------------- */
 typedef enum { ROCS_NORM_NONE = 0, ROCS_NORM_LAYER = 1, ROCS_NORM_RMS = 2 } rocs_norm;
 typedef enum { ROCS_ACT_NONE = 0, ROCS_ACT_RELU = 1, ROCS_ACT_SILU = 2, ROCS_ACT_GELU = 3 } rocs_act;
@@ -358,7 +359,7 @@ ROCS_API int rocs_proj_forward(const rocs_proj_args* args, rocs_stream_t stream)
  *   q     [C, n_out] bf16 out: the candidate queries (input of rocs_dca_forward)
  *   Shapes as rocs_lcb_forward (ROCS_BF16) with o_r + o_c in place of o_r, n_out % 256 == 0,
  *   (n_c*d) % 64 == 0.  Workspace rocs_chain_split_workspace_size(); one status header for all
- *   steps (rocs_read_status).  Three kernel launches plus memsets.
+ *   steps (rocs_read_status).  Four kernel launches plus memsets.
  * ---------------------------------------------------------------------------------- */
 typedef struct {
   int64_t n_out, o_r, o_c, n_r, n_c, d;
