@@ -656,15 +656,16 @@ template <int DH>
 static cudaError_t launch_t(const DcaParams& p, int grid, cudaStream_t st) {
   using L = DcaSmem<DH>;
   auto k = rocs_dca_sm100_kernel<DH>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static std::atomic<uint64_t> optin_done{0};  // one bit per device
+  static std::atomic<int> regs_checked{0};       // a property of the binary: checked once per process
+  if (!regs_checked.load(std::memory_order_acquire)) {
     // the setmaxnreg split is only valid for the register count it was computed for
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, k) != cudaSuccess || fa.numRegs != (int)kLaunchRegs) return cudaErrorInvalidConfiguration;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::alloc_bytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+    regs_checked.store(1, std::memory_order_release);
   }
+  cudaError_t e = ensure_smem_optin(optin_done, k, (int)L::alloc_bytes);
+  if (e != cudaSuccess) return e;
   // programmatic dependent launch: set-up (barriers, TMEM, descriptor prefetch) overlaps the scheduling
   // kernel that precedes it on the stream
   return launch_dependent(k, grid, kThreads, L::alloc_bytes, st, p);

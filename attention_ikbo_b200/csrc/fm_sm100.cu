@@ -364,12 +364,9 @@ template <int D>
 static cudaError_t launch_t(const FmParams& p, int grid, cudaStream_t st) {
   using L = FmSmem<D>;
   auto k = rocs_fm_sm100_kernel<D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::alloc_bytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> optin_done{0};  // per instantiation, one bit per device
+  cudaError_t e = ensure_smem_optin(optin_done, k, (int)L::alloc_bytes);
+  if (e != cudaSuccess) return e;
   return launch_dependent(k, grid, kThreads, L::alloc_bytes, st, p);
 }
 

@@ -605,12 +605,9 @@ static cudaError_t launch_t(const LcbParams& p, int grid, cudaStream_t st) {
   constexpr int NG = EPI_C >= 0 ? 2 : 1;
   using L = LcbSmem<D, NC, NG>;
   auto k = rocs_lcb_sm100_kernel<D, NC, EPI_C, NG>;
-  static bool attr_set = false;  // per instantiation; harmless if two threads race
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::alloc_bytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> optin_done{0};  // per instantiation, one bit per device
+  cudaError_t e = ensure_smem_optin(optin_done, k, (int)L::alloc_bytes);
+  if (e != cudaSuccess) return e;
   return launch_dependent(k, grid, LcbRoles<NG>::kThreads, L::alloc_bytes, st, p);
 }
 

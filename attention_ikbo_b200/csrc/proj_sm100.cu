@@ -202,13 +202,9 @@ cudaError_t launch_chain_fold(const __nv_bfloat16* w_q, const __nv_bfloat16* w_c
 }
 
 cudaError_t launch_proj_sm100(const ProjParams& p, int grid, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(rocs_proj_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)alloc_bytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> optin_done{0};  // one bit per device
+  cudaError_t e = ensure_smem_optin(optin_done, rocs_proj_sm100_kernel, (int)alloc_bytes);
+  if (e != cudaSuccess) return e;
   rocs_proj_sm100_kernel<<<grid, kThreads, alloc_bytes, st>>>(p);
   return cudaGetLastError();
 }

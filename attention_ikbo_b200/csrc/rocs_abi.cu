@@ -372,6 +372,10 @@ int dca_run_ext(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, W
 size_t dca_body_bytes_ext(int64_t R, int64_t n_units) { return dca_body(R, n_units).body; }
 int64_t dca_units_ext(const rocs_dca_args* a) { return dca_units(a); }
 void set_last_launches(int n) { g_last_launches = n; }
+std::atomic<uint64_t>& configured_device_mask_ref() {
+  static std::atomic<uint64_t> mask{0};
+  return mask;
+}
 }  // namespace rocs
 
 extern "C" {
@@ -856,5 +860,7 @@ const char* rocs_status_string(int code) {
 }
 
 int rocs_last_launch_count(void) { return g_last_launches; }
+
+uint64_t rocs_configured_device_mask(void) { return configured_device_mask_ref().load(std::memory_order_acquire); }
 
 }  // extern "C"

@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "rocs_ikbo.h"
 
 namespace rocs {
@@ -293,6 +295,29 @@ __device__ __forceinline__ void reg_alloc() {
 template <uint32_t N>
 __device__ __forceinline__ void reg_dealloc() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ------------------------------------------------------------------ host: per-device kernel set-up
+// cudaFuncSetAttribute (the opt-in to more than 48 KB of dynamic shared memory) applies to the CURRENT
+// device only, so whether it has been done is tracked per device: one bit per device ordinal in an
+// atomic mask per kernel.  A process that drives several GPUs sets the attribute once on each.
+// Devices past ordinal 63 are set up on every call (correct, just not cached).  Every bit that is set
+// is also recorded in a library-wide mask that rocs_configured_device_mask() reports.
+std::atomic<uint64_t>& configured_device_mask_ref();
+template <typename Kernel>
+inline cudaError_t ensure_smem_optin(std::atomic<uint64_t>& done, Kernel kernel, int smem_bytes) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t{1} << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e != cudaSuccess) return e;
+  if (bit) {
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    configured_device_mask_ref().fetch_or(bit, std::memory_order_acq_rel);
+  }
+  return cudaSuccess;
 }
 
 // ------------------------------------------------------------------ host: dependent launch

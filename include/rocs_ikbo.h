@@ -147,11 +147,21 @@ ROCS_API int rocs_lcb_forward_fault_injection(const rocs_lcb_args* args, rocs_st
  *     must be serialised by the caller.  The array keeps the last call's contents; each
  *     call clears the status word and flags itself.
  *   - The first call on a device looks up the array's device address (once per device);
- *     make that first call before any stream capture starts.
- *   - Device-side status is kept in the array's own header and is not readable through
- *     rocs_read_status(); host-side validation errors are returned as for rocs_lcb_forward. */
+ *     make that first call before any stream capture starts.  cudaDeviceReset() invalidates
+ *     that address: do not use this entry point on a device after resetting it.
+ *   - Device-side status (a bounded wait that expired: ROCS_ERR_TIMEOUT; a bad device
+ *     offset: ROCS_ERR_DEVICE_INDEX) is kept in the array's own header: read it with
+ *     rocs_lcb_noalloc_read_status(), not rocs_read_status().  Host-side validation errors
+ *     are returned as for rocs_lcb_forward. */
 #define ROCS_LCB_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 ROCS_API int rocs_lcb_forward_noalloc(const rocs_lcb_args* args, rocs_stream_t stream);
+
+/* Device status of the last rocs_lcb_forward_noalloc call on the CURRENT device (the paper
+ * has no counterpart).  Synchronises `stream`, then copies the code and detail words from the
+ * header of the library's scratch array into *device_code (a rocs_status; required) and
+ * *detail (may be NULL); allocates nothing.  Call it on the stream of that call, with the same
+ * device current.  Returns ROCS_OK, or ROCS_ERR_INVALID_ARG / ROCS_ERR_CUDA for the read. */
+ROCS_API int rocs_lcb_noalloc_read_status(rocs_stream_t stream, int32_t* device_code, int32_t* detail);
 
 /* ------------------------------------------------------------------------------------
  * LCB block: IKBO-LCB with a fused per-group output epilogue
@@ -432,6 +442,13 @@ ROCS_API const char* rocs_status_string(int code);
 /* Number of kernel launches the last successful *_forward call on this host thread
  * enqueued (memsets not counted). */
 ROCS_API int rocs_last_launch_count(void);
+
+/* Bit k is set once some kernel of this library has had its per-device set-up (the opt-in to
+ * large dynamic shared memory, which CUDA applies to the current device only) done on device
+ * ordinal k in this process.  The set-up runs on the first launch of each kernel on each device,
+ * so a process that drives several GPUs configures every one of them.  Ordinals past 63 are
+ * configured on every launch and not recorded.  Host-only; never fails. */
+ROCS_API uint64_t rocs_configured_device_mask(void);
 
 #ifdef __cplusplus
 }

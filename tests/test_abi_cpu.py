@@ -214,3 +214,15 @@ def test_host_pipeline_host_validation(lib):
     assert lib.rocs_lcb_forward_host(P(a), 2, None, need, None) == 6
     bad, keep2 = _lcb_args(m, [0, 3, 2])
     assert lib.rocs_lcb_forward_host(P(bad), 2, 0x10000, need, None) == 2
+
+
+def test_configured_device_mask_starts_empty(lib):
+    """The per-device kernel set-up is recorded per device ordinal; nothing is configured before a
+    launch (and nothing can be without a GPU).  Host-only query; the GPU side is in test_gpu_edges."""
+    lib.rocs_configured_device_mask.restype = ctypes.c_uint64
+    assert lib.rocs_configured_device_mask() == 0
+
+
+def test_noalloc_status_reader_rejects_null(lib):
+    lib.rocs_lcb_noalloc_read_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    assert lib.rocs_lcb_noalloc_read_status(None, None, None) == 1  # ROCS_ERR_INVALID_ARG, before any CUDA call

@@ -105,3 +105,20 @@ def test_chain_full_size_sampled(ikbo, oracle_mod):
     assert_close(host_f64(y_cand[idx]), yc, "bf16", "Y^C")
     assert_close(host_f64(o[idx]).reshape(oo.shape), oo, "bf16", "O")
     assert_close(host_f64(lse[idx]).reshape(ll.shape), ll, "bf16", "LSE")
+
+
+def test_kernel_setup_recorded_for_the_device_used(ikbo, oracle_mod):
+    """cudaFuncSetAttribute applies to the current device only: the library records its per-kernel
+    set-up per device ordinal.  After launches on this device, its bit is set (and only bits of
+    devices this process has used)."""
+    import ctypes
+
+    lib = ikbo.load_library()
+    lib.rocs_configured_device_mask.restype = ctypes.c_uint64
+    x = ri.make_lcb("m", [4, 9], 256, 64, 128, 128, 128, 82, "bf16")
+    ikbo.rocs_lcb_forward(*[dev(a) for a in (x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)], x.cand_off)
+    status_ok(ikbo, ikbo.rocs_lcb_forward.last_workspace)
+    mask = int(lib.rocs_configured_device_mask())
+    d = torch.cuda.current_device()
+    assert mask & (1 << d), hex(mask)
+    assert mask >> torch.cuda.device_count() == 0, hex(mask)
