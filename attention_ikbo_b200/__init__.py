@@ -49,6 +49,7 @@ from ._binding import (  # noqa: F401
     rocs_lcb_forward_fault_injection,
     rocs_lcb_forward_host,
     rocs_lcb_forward_noalloc,
+    rocs_lcb_noalloc_read_status,
     rocs_pad_cols,
     rocs_proj_forward,
     rocs_read_status,

@@ -111,7 +111,8 @@ def load_library():
                            ("rocs_chain_prepare_weights", [P(ChainWeightsArgs), _vp]),
                            ("rocs_chain_split_forward", [P(ChainSplitArgs), _vp]),
                            ("rocs_pad_cols", [_vp, _i64, _i64, _i64, _vp, _i64, _i64, _vp]),
-                           ("rocs_read_status", [_vp, _vp, P(_i32), P(_i32)])]:
+                           ("rocs_read_status", [_vp, _vp, P(_i32), P(_i32)]),
+                           ("rocs_lcb_noalloc_read_status", [_vp, P(_i32), P(_i32)])]:
             getattr(lib, name).restype = ctypes.c_int
             getattr(lib, name).argtypes = argt
         for name, argt in [("rocs_lcb_host_staging_size", [P(LcbArgs), _i64]),
@@ -227,12 +228,29 @@ def rocs_lcb_forward_noalloc(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y
 
     Uses the library's fixed device scratch array instead of a workspace (see the header for its
     size limit and for why concurrent calls on one device must be serialised).  ``y_req`` and
-    ``y_cand`` must be given: this call allocates nothing.
+    ``y_cand`` must be given: this call allocates nothing.  ``cand_off`` should be the pair from
+    ``offsets()`` so that no offsets tensor is created either.  The call runs with the device of
+    ``x_req`` current, so the scratch array it uses is that device's.  Read its device status with
+    ``rocs_lcb_noalloc_read_status``.
     """
+    if y_req is None or y_cand is None:
+        raise RocsError(1, "rocs_lcb_forward_noalloc: y_req and y_cand must be given (this call allocates nothing)")
     lib = load_library()
-    a, keep, y_req, y_cand = _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y_cand)
-    _check(lib.rocs_lcb_forward_noalloc(ctypes.byref(a), _stream(stream)), "rocs_lcb_forward_noalloc")
+    with torch.cuda.device(x_req.device):
+        a, keep, y_req, y_cand = _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y_cand)
+        _check(lib.rocs_lcb_forward_noalloc(ctypes.byref(a), _stream(stream)), "rocs_lcb_forward_noalloc")
     return y_req, y_cand
+
+
+def rocs_lcb_noalloc_read_status(device=None, stream=None):
+    """Synchronise the stream and return ``(device_code, detail)`` of the last no-alloc LCB call on
+    ``device`` (default: the current device)."""
+    lib = load_library()
+    code, detail = ctypes.c_int32(0), ctypes.c_int32(0)
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        _check(lib.rocs_lcb_noalloc_read_status(_stream(stream), ctypes.byref(code), ctypes.byref(detail)),
+               "rocs_lcb_noalloc_read_status")
+    return code.value, detail.value
 
 
 def rocs_lcb_forward_fault_injection(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, skip_release_request,

@@ -20,9 +20,14 @@
 //     start at zero (status word and ready flags) before its kernel runs;
 //   * the first call on a device looks up the array's device address (cudaGetSymbolAddress,
 //     once per device, with that device current).  Make that first call before any stream
-//     capture begins;
-//   * device-side status (a bounded wait that expired) is recorded in the array's own header,
-//     which rocs_read_status() cannot reach; host-side validation errors are returned as usual.
+//     capture begins.  cudaDeviceReset() unloads the library's device code, so the looked-up
+//     address is stale afterwards: do not call this entry point after resetting a device that
+//     it has already run on;
+//   * device-side status (a bounded wait that expired, a bad device offset) is recorded in the
+//     array's own header; rocs_lcb_noalloc_read_status() reads it without allocating.  Host-side
+//     validation errors are returned as usual.
+#include <atomic>
+
 #include "lcb_sm100.h"
 
 namespace rocs {
@@ -44,19 +49,21 @@ static_assert(kNoallocScratchBytes % 256 == 0, "scratch size is a multiple of 25
 static __device__ __align__(256) uint8_t g_lcb_noalloc_scratch[kNoallocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
+// One slot per device ordinal.  Atomic, so host threads that make their first call at the same time
+// may both look the address up, but each reads and publishes a complete pointer (the same one).
+std::atomic<void*> g_scratch_addr[kMaxDevices];
 
 // Device address of the array on the current device (looked up once per device).
 int scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return ROCS_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return ROCS_ERR_UNSUPPORTED;
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
+  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
     if (cudaGetSymbolAddress(&p, g_lcb_noalloc_scratch) != cudaSuccess || p == nullptr) return ROCS_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    g_scratch_addr[dev].store(p, std::memory_order_release);
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return ROCS_OK;
 }
 
@@ -76,4 +83,18 @@ extern "C" int rocs_lcb_forward_noalloc(const rocs_lcb_args* a, rocs_stream_t st
   rc = lcb_run_ext(a, C, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream), &launches);
   if (rc == ROCS_OK) set_last_launches(launches);
   return rc;
+}
+
+extern "C" int rocs_lcb_noalloc_read_status(rocs_stream_t stream, int32_t* device_code, int32_t* detail) {
+  if (!device_code) return ROCS_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc) return rc;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t h[2] = {0, 0};  // code and detail: the first 8 bytes of the header at the start of the array
+  if (cudaMemcpyAsync(h, scratch, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return ROCS_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ROCS_ERR_CUDA;
+  *device_code = h[0];
+  if (detail) *detail = h[1];
+  return ROCS_OK;
 }
