@@ -616,7 +616,7 @@ def make_parts(workload):
     if workload == "dca_expand":
         return [DcaExpandPart(ri.dca_long())]
     if workload == "chain":
-        ci = ri.chain()
+        ci = _CHAIN.get("ci") or ri.chain()
         lcb = LcbPart(ci.lcb, "chain_lcb")
         x = ci.lcb
         qdummy = np.zeros((0,), np.uint16)
@@ -624,7 +624,7 @@ def make_parts(workload):
         _CHAIN["ci"] = ci
         return [lcb, ProjPart(ci, lcb), DcaPart(dca_in, "chain_dca")]
     if workload == "chain_split":
-        ci = ri.chain()
+        ci = _CHAIN.get("ci") or ri.chain()
         x = ci.lcb
         qdummy = np.zeros((0,), np.uint16)
         dca_in = ri.DcaInputs("chain_dca", x.cand_off, ci.seq_off, 1, ci.H, ci.dh, ci.scale, qdummy, ci.k_t, ci.v_t)
@@ -786,26 +786,138 @@ def run_reference(args):
         t, f = p.oracle_sample(oracle, 1, 7 + i)
         unit_t.append(t)
     ns = [int(max(1, min(4096, per_step_budget / len(oparts) / max(t, 1e-6)))) for t in unit_t]
-    vals, times = [], []
+    vals, times, walls, fracs = [], [], [], []
     for k in range(args.warmup + args.steps):
-        est = 0.0
+        est, wall, cover = 0.0, 0.0, []
         for i, p in enumerate(oparts):
             t, f = p.oracle_sample(oracle, ns[i], 1000 * k + i)
             est += t / f
+            wall += t
+            cover.append(f)
         if k >= args.warmup:
             times.append(est)
+            walls.append(wall)
+            fracs.append(cover)
             vals.append(step_flops / est / 1e12)
     value = float(statistics.mean(vals))
     sample = "; ".join(f"{p.name}: {n} random candidates per step, scaled by the work they cover"
                        for p, n in zip(oparts, ns))
     cores = oracle.max_threads()
+    cfg = workload_config(args.workload, parts)
+    # the other workloads, on rank 0 of a single-GPU run only (a multi-GPU run holds every GPU meanwhile)
+    reported = None
+    if world == 1 and args.workload == "ikbo_step" and not args.no_reported:
+        parts = p = None  # the headline step's device buffers
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        reported = run_reported(ikbo, torch, dev, flush, max(3, min(args.warmup, 5)), peaks, peak_src,
+                                args.no_clocks)
+
+    cfg.update({"parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU",
+                "l2": "flushed between timed steps (256 MiB write outside the per-step CUDA events)"})
+    # Each step times the oracle on a random sample of candidates and scales it to the whole step by the
+    # fraction of the step's work the sample covers: ms_per_step is that extrapolation, sampled_ms_per_step
+    # the wall-clock the sample itself took.
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(statistics.mean(times)),
+            "extrapolated": True, "sampled_ms_per_step": 1e3 * float(statistics.mean(walls)),
+            "sampled_candidates_per_step": {p.name: n for p, n in zip(oparts, ns)},
+            "sampled_fraction_per_step": {p.name: float(statistics.mean(c[i] for c in fracs))
+                                          for i, p in enumerate(oparts)},
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(args.workload, parts),
+            "config": cfg,
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
+
+
+def parts_to_device(workload, parts, ikbo, torch, dev):
+    """Inputs of every part resident on `dev` (the chained workloads feed one part's output to the next)."""
+    for p in parts:
+        if isinstance(p, DcaPart) and workload == "chain":
+            p.to_device(ikbo, torch, dev, q_dev=parts[1].out)
+        elif isinstance(p, DcaPart) and workload == "chain_split":
+            p.to_device(ikbo, torch, dev, q_dev=parts[0].out)
+        else:
+            p.to_device(ikbo, torch, dev)
+    torch.cuda.synchronize()
+
+
+def check_status(parts, ikbo):
+    for p in parts:
+        code, detail = p.status(ikbo)
+        if code != 0:
+            raise SystemExit(f"{p.name}: device status {ikbo.STATUS_NAMES.get(code)} at {detail}")
+
+
+def timed_steps(parts, ikbo, torch, steps, flush, stream):
+    """`steps` steps, each after an L2 flush (outside the events); per part the mean CUDA-event time in ms
+    (events on the launching stream) and the number of kernels launched."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(steps)]
+    launches = 0
+    for k in range(steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        for j, p in enumerate(parts):
+            launches += p.run(ikbo)
+            ev[k][j + 1].record(stream)
+    torch.cuda.synchronize()
+    part_ms = [statistics.mean(ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(steps))
+               for j in range(len(parts))]
+    return part_ms, launches
+
+
+def roofline_row(p, ms, peaks, peak_src):
+    sec = ms * 1e-3
+    if p.bound == "hbm":
+        ach, peak, unit = p.bytes() / sec / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        ach, peak, unit = p.flops() / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    return {"kernel": p.name, "bound": p.bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+            "traffic": ncu_traffic(p), "peak_source": f"{peak_src} (burst)"}
+
+
+# Workloads timed after the headline step and reported beside it (steps each; the explicit-expand
+# baselines are timed on the same inputs as their IKBO workloads and counted on the IKBO work).
+REPORTED = [("dca_short", 30), ("dca_block", 20), ("lcb_block", 30), ("fm", 30), ("chain", 10), ("chain_split", 10),
+            ("lcb_expand", 10), ("dca_expand", 3)]
+
+
+def run_reported(ikbo, torch, dev, flush, warmup, peaks, peak_src, no_clocks):
+    """Every other workload, one after another (inputs freed in between), timed like the headline step."""
+    out = []
+    stream = torch.cuda.current_stream()
+    for wl, steps in REPORTED:
+        parts = make_parts(wl)
+        parts_to_device(wl, parts, ikbo, torch, dev)
+        check_status(parts, ikbo)
+        for _ in range(warmup):
+            flush.zero_()
+            for p in parts:
+                p.run(ikbo)
+        torch.cuda.synchronize()
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        sampler = None if no_clocks else ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        if sampler is not None:
+            time.sleep(0.2)
+        part_ms, launches = timed_steps(parts, ikbo, torch, steps, flush, stream)
+        clocks = sampler.stop() if sampler is not None else None
+        check_status(parts, ikbo)
+        rows = []
+        for p, ms in zip(parts, part_ms):
+            r = roofline_row(p, ms, peaks, peak_src)
+            r.update({"ms": ms, "tflops": p.flops() / (ms * 1e-3) / 1e12, "gbs": p.bytes() / (ms * 1e-3) / 1e9,
+                      "candidates_per_s": p.units / (ms * 1e-3)})
+            rows.append(r)
+        step_ms = sum(part_ms)
+        out.append({"workload": wl, "steps": steps, "warmup": warmup, "ms_per_step": step_ms,
+                    "value": sum(p.flops() for p in parts) / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "config": workload_config(wl, parts), "parts": rows, "gpu_launches": launches,
+                    "clocks": clocks})
+        del parts
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ikbo(args):
@@ -828,18 +940,8 @@ def run_ikbo(args):
     ikbo.load_library()
 
     parts = make_parts(args.workload)
-    for p in parts:
-        if isinstance(p, DcaPart) and args.workload == "chain":
-            p.to_device(ikbo, torch, dev, q_dev=parts[1].out)
-        elif isinstance(p, DcaPart) and args.workload == "chain_split":
-            p.to_device(ikbo, torch, dev, q_dev=parts[0].out)
-        else:
-            p.to_device(ikbo, torch, dev)
-    torch.cuda.synchronize()
-    for p in parts:
-        code, detail = p.status(ikbo)
-        if code != 0:
-            raise SystemExit(f"{p.name}: device status {ikbo.STATUS_NAMES.get(code)} at {detail}")
+    parts_to_device(args.workload, parts, ikbo, torch, dev)
+    check_status(parts, ikbo)
 
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # 256 MiB > 126 MB L2
     stream = torch.cuda.current_stream()
@@ -865,26 +967,12 @@ def run_ikbo(args):
     sampler = None if args.no_clocks else ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
     if sampler is not None:
         time.sleep(0.3)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(args.steps)]
-    launches = 0
-    for k in range(args.steps):
-        flush.zero_()  # L2 flush between steps, outside the per-step events
-        ev[k][0].record(stream)
-        for j, p in enumerate(parts):
-            launches += p.run(ikbo)
-            ev[k][j + 1].record(stream)
-    torch.cuda.synchronize()
+    part_ms, launches = timed_steps(parts, ikbo, torch, args.steps, flush, stream)
     barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler is not None else None
-
-    part_ms = [statistics.mean(ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(args.steps))
-               for j in range(len(parts))]
     step_ms = sum(part_ms)
-    for p in parts:
-        code, detail = p.status(ikbo)
-        if code != 0:
-            raise SystemExit(f"{p.name}: device status {ikbo.STATUS_NAMES.get(code)} at {detail}")
+    check_status(parts, ikbo)
     step_ms = reduce_max(step_ms, dist, dev)
 
     # ---- end to end through the public API: pinned host inputs -> device -> kernels -> host outputs.
@@ -947,13 +1035,7 @@ def run_ikbo(args):
     rooflines, part_rows = [], []
     for p, ms in zip(parts, part_ms):
         sec = ms * 1e-3
-        if p.bound == "hbm":
-            ach, peak, unit = p.bytes() / sec / 1e9, peaks["hbm_gbs"], "GB/s"
-        else:
-            ach, peak, unit = p.flops() / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-        rf = {"kernel": p.name, "bound": p.bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
-              "traffic": ncu_traffic(p), "peak_source": f"{peak_src} (burst)"}
-        rooflines.append(rf)
+        rooflines.append(roofline_row(p, ms, peaks, peak_src))
         part_rows.append({"name": p.name, "ms": ms, "tflops": p.flops() / sec / 1e12, "gbs": p.bytes() / sec / 1e9,
                           "candidates_per_s": p.units / sec, "algorithmic_flops": p.flops(),
                           "algorithmic_bytes": p.bytes()})
@@ -980,6 +1062,8 @@ def run_ikbo(args):
             "roofline": {k: v for k, v in rooflines[dom].items()}, "rooflines": rooflines, "parts": part_rows,
             "candidates_per_s": {r["name"]: r["candidates_per_s"] for r in part_rows},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
+    if reported is not None:
+        line["reported"] = reported
     print(json.dumps(line))
 
 
@@ -997,6 +1081,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-reported", action="store_true",
+                    help="skip timing the other workloads after the default step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
