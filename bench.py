@@ -804,15 +804,6 @@ def run_reference(args):
                        for p, n in zip(oparts, ns))
     cores = oracle.max_threads()
     cfg = workload_config(args.workload, parts)
-    # the other workloads, on rank 0 of a single-GPU run only (a multi-GPU run holds every GPU meanwhile)
-    reported = None
-    if world == 1 and args.workload == "ikbo_step" and not args.no_reported:
-        parts = p = None  # the headline step's device buffers
-        torch.cuda.synchronize()
-        torch.cuda.empty_cache()
-        reported = run_reported(ikbo, torch, dev, flush, max(3, min(args.warmup, 5)), peaks, peak_src,
-                                args.no_clocks)
-
     cfg.update({"parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU",
                 "l2": "flushed between timed steps (256 MiB write outside the per-step CUDA events)"})
     # Each step times the oracle on a random sample of candidates and scales it to the whole step by the
@@ -1054,6 +1045,15 @@ def run_ikbo(args):
                                  "est_seconds_per_step": est1}}
 
     cfg = workload_config(args.workload, parts)
+    # the other workloads, on rank 0 of a single-GPU run only (a multi-GPU run holds every GPU meanwhile)
+    reported = None
+    if world == 1 and args.workload == "ikbo_step" and not args.no_reported:
+        parts = p = None  # the headline step's device buffers
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        reported = run_reported(ikbo, torch, dev, flush, max(3, min(args.warmup, 5)), peaks, peak_src,
+                                args.no_clocks)
+
     cfg.update({"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                 "l2": "flushed between timed steps (256 MiB write outside the per-step CUDA events)"})
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
