@@ -54,10 +54,12 @@ constexpr int kRowsPerUnit = 2 * BM;
 template <int DH>
 struct DcaSmem {
   static constexpr uint32_t kTile = BM * DH * 2;  // one Q tile or one K/V tile (bf16)
-  static constexpr int kRing = DH == 128 ? 5 : 10;
+  static constexpr int kRing = DH == 128 ? 4 : 10;
+  static constexpr uint32_t kStage = 32 * 128;     // per softmax warp: 32 rows x 64 columns of O (bf16)
   static constexpr uint32_t off_q = 0;
   static constexpr uint32_t off_ring = 2 * kTile;
-  static constexpr uint32_t off_bar = off_ring + kRing * kTile;
+  static constexpr uint32_t off_stage = off_ring + kRing * kTile;  // 8 warps x kStage, 1024-byte aligned
+  static constexpr uint32_t off_bar = off_stage + 8 * kStage;
   static constexpr uint32_t n_bars = 2 * kRing + 2 * 8 + 1 + 4;
   static constexpr uint32_t off_misc = off_bar + n_bars * 8;
   static constexpr uint32_t bytes = off_misc + 64;
@@ -127,6 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_q = smem + L::off_q;
   uint8_t* s_ring = smem + L::off_ring;
+  uint8_t* s_stage = smem + L::off_stage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::off_bar);
   uint64_t* ring_full = bars;
   uint64_t* ring_empty = bars + kRing;
@@ -400,6 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
     const uint32_t s_addr = tmem_base + t_lane + x * 128;
     const uint32_t p_addr = kSepP ? tmem_base + t_lane + kPCol + x * 64 : s_addr;
     const uint32_t o_addr = tmem_base + t_lane + 256 + x * DH;
+    uint8_t* stage = s_stage + (warp - kSoftmaxWarp0) * L::kStage;  // this warp's O staging slab
+    const uint32_t stage_a = smem_u32(stage);
     const float c = p.scale_log2;
     uint32_t ws_ = 0, wph = 0, sph = 0, ofph = 0, n_sig = 0;
     bool ok = true;
@@ -552,19 +557,46 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       ofph ^= 1;
       tc_fence_after();
       const float inv = 1.0f / l;
+      // This warp's 32 rows of the tile.  A full slab leaves through its shared-memory slab and a TMA store,
+      // one 64-column box at a time: a handful of instructions per warp, where row-by-row 16-byte stores
+      // (32 rows apart per instruction) would queue thousands of small writes in the SM's memory pipeline, in
+      // front of the producer's and the issuer's own memory instructions.  A slab cut by the end of the
+      // request's rows is stored row by row, so that no row of the next request is written.
+      const int slab0 = w.row0 + x * BM + 32 * quarter;  // first row of the slab within the request
+      const bool tma_slab = slab0 + 32 <= w.rows;
 #pragma unroll 1
-      for (int cc = 0; cc < DH / 32; ++cc) {
-        uint32_t ov[32];
-        tmem_ld32(o_addr + cc * 32, ov);
-        tmem_ld_wait();
-        if (row_ok) {
+      for (int cc = 0; cc < DH / 64; ++cc) {
+        uint32_t ov[2][32];
+        tmem_ld32(o_addr + cc * 64, ov[0]);
+        tmem_ld32(o_addr + cc * 64 + 32, ov[1]);
+        tmem_ld_wait_regs(ov[0], ov[1]);
+        if (tma_slab) {
+          if (lane == 0) bulk_wait_read<0>();  // the slab's previous store has finished reading it
+          __syncwarp();
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            st_global_v4(orow + cc * 32 + 8 * k,
-                         pack_bf16x2(__uint_as_float(ov[8 * k + 0]) * inv, __uint_as_float(ov[8 * k + 1]) * inv),
-                         pack_bf16x2(__uint_as_float(ov[8 * k + 2]) * inv, __uint_as_float(ov[8 * k + 3]) * inv),
-                         pack_bf16x2(__uint_as_float(ov[8 * k + 4]) * inv, __uint_as_float(ov[8 * k + 5]) * inv),
-                         pack_bf16x2(__uint_as_float(ov[8 * k + 6]) * inv, __uint_as_float(ov[8 * k + 7]) * inv));
+          for (int c16 = 0; c16 < 8; ++c16) {  // row `lane`: 8 chunks of 16 bytes, 128-byte swizzle
+            const uint32_t* v = &ov[c16 >> 2][(c16 & 3) * 8];
+            st_shared_v4(stage_a + lane * 128 + ((c16 ^ (lane & 7)) << 4),
+                         pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
+                         pack_bf16x2(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
+                         pack_bf16x2(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
+                         pack_bf16x2(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&p.tm_o, stage, w.h * DH + cc * 64, w.qbase + slab0);
+            bulk_commit();
+          }
+        } else if (row_ok) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t* v = &ov[k >> 2][(k & 3) * 8];
+            st_global_v4(orow + cc * 64 + 8 * k, pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv),
+                         pack_bf16x2(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv),
+                         pack_bf16x2(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv),
+                         pack_bf16x2(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv));
+          }
         }
       }
       tc_fence_before();
@@ -573,6 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       if (row_ok && p.lse) p.lse[(size_t)(w.qbase + row) * p.H + w.h] = (m_used + lg2(l)) * 0.69314718055994531f;
     }
     (void)ok;
+    if (lane == 0) bulk_wait<0>();  // every TMA store of this warp has completed
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -45,6 +45,7 @@ struct DcaParams {
   CUtensorMap tm_q;  // Q viewed as [C*q, H*dh], box {64, 128}
   CUtensorMap tm_k;  // K viewed as [T, H*dh],   box {64, 128}
   CUtensorMap tm_v;  // V viewed as [T, H*dh],   box {64, 128}
+  CUtensorMap tm_o;  // O viewed as [C*q, H*dh], box {64, 32}   (stores)
   const int32_t* cand_off;
   const int32_t* seq_off;
   const int4* units;  // work-unit table {r, h, row0, 0}

@@ -329,6 +329,7 @@ int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHea
   std::memset(&p, 0, sizeof(p));
   const uint64_t hd = a->H * a->dh, rb = hd * 2, kvb = (a->kv_ld ? a->kv_ld : hd) * 2;
   bool ok = tmap_bf16(&p.tm_q, a->q_ptr, hd, (uint64_t)C * a->q, rb, 64, 128);
+  ok &= tmap_bf16(&p.tm_o, a->o_ptr, hd, (uint64_t)C * a->q, rb, 64, 32);
   if (T > 0) {
     ok &= tmap_bf16(&p.tm_k, a->k_ptr, hd, (uint64_t)T, kvb, 64, 128);
     ok &= tmap_bf16(&p.tm_v, a->v_ptr, hd, (uint64_t)T, kvb, 64, 128);
