@@ -66,5 +66,9 @@ def test_split_chain_full_size_sampled(ikbo, oracle_mod):
     request outputs in full, a seeded sample of candidates."""
     ci = ri.chain()
     _, _, y_req, q, o, lse = run_split(ikbo, ci)
-    sel = np.unique(ri.uniform_int(19, 1, 0, ci.lcb.C - 1, 24).astype(np.int64))
+    # 520 random candidates plus the first and last of every request (about 0.75 % of ~100k)
+    off = np.asarray(ci.lcb.cand_off).astype(np.int64)
+    ends = [c for r in range(ci.lcb.R) if off[r + 1] > off[r] for c in (off[r], off[r + 1] - 1)]
+    sel = np.unique(np.concatenate([ri.uniform_int(19, 1, 0, ci.lcb.C - 1, 520).astype(np.int64), ends]))
+    assert len(sel) >= 0.005 * ci.lcb.C
     check(oracle_mod, ci, y_req, q, o, lse, sel)

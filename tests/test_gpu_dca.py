@@ -104,17 +104,25 @@ def _sample(x, n, seed):
 
 
 def test_dca_bf16_full_size_sampled(ikbo, oracle_mod):
-    """R=32, L=2048, H=8, dh=128, 512 candidates per request, q=1."""
+    """R=32, L=2048, H=8, dh=128, 512 candidates per request, q=1: 200 random candidates plus the first and
+    last of every request (1.6 % of the 16,384)."""
     x = ri.dca_bf16()
     o, lse = run_dca(ikbo, x)
-    check(oracle_mod, x, o, lse, sel=_sample(x, 64, 2))
+    sel = _sample(x, 200, 2)
+    assert len(sel) >= 0.01 * x.C
+    check(oracle_mod, x, o, lse, sel=sel)
 
 
 def test_dca_long_full_size_sampled(ikbo, oracle_mod):
-    """R=8, L_r~U{4096..8192}, H=4, dh=128, 2048 candidates per request, q=4."""
+    """R=8, L_r~U{4096..8192}, H=4, dh=128, 2048 candidates per request, q=4: 168 random candidates plus the
+    first and last of every request (over 1 % of the 16,384, every request represented)."""
     x = ri.dca_long()
     o, lse = run_dca(ikbo, x)
-    check(oracle_mod, x, o, lse, sel=_sample(x, 24, 3))
+    sel = _sample(x, 168, 3)
+    assert len(sel) >= 0.01 * x.C
+    off = np.asarray(x.cand_off)
+    assert all(((sel >= off[r]) & (sel < off[r + 1])).any() for r in range(x.R))
+    check(oracle_mod, x, o, lse, sel=sel)
 
 
 def _f32_to_bf16(a):

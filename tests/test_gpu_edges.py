@@ -99,7 +99,11 @@ def test_chain_full_size_sampled(ikbo, oracle_mod):
     y_req, y_cand, q, o, lse = ikbo.chain_forward(*[dev(a) for a in (x.x_req, x.x_cand, x.w_rr, x.w_cr, x.w_cc)],
                                                   x.cand_off, dev(ci.w_q), dev(ci.k_t), dev(ci.v_t), ci.seq_off,
                                                   ci.H, ci.dh, ci.scale)
-    sel = np.unique(ri.uniform_int(23, 1, 0, x.C - 1, 16).astype(np.int64))
+    # 520 random candidates plus the first and last of every request (about 0.75 % of ~100k)
+    off = np.asarray(x.cand_off).astype(np.int64)
+    ends = [c for r in range(x.R) if off[r + 1] > off[r] for c in (off[r], off[r + 1] - 1)]
+    sel = np.unique(np.concatenate([ri.uniform_int(23, 1, 0, x.C - 1, 520).astype(np.int64), ends]))
+    assert len(sel) >= 0.005 * x.C
     yc, qo, oo, ll = oracle_mod.chain(ci, sel)
     idx = torch.as_tensor(sel, device=q.device)
     assert_close(host_f64(y_cand[idx]), yc, "bf16", "Y^C")
