@@ -191,7 +191,11 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
         if (!mbar_wait(&empty[s], ph ^ 1, ctl, 103)) { ok = false; break; }
         uint8_t* slot = s_ring + s * kSlot;
         mbar_arrive_expect_tx(&full[s], L::kXc);
-        for (int cc = 0; cc < D / 64; ++cc) tma_load_2d(slot + cc * (NC * 128), &p.tm_xc, &full[s], cc * 64, i * NC);
+        for (int cc = 0; cc < D / 64; ++cc) {
+          // LCB block: X^C is read once; evict-first keeps the residual rows prefetched for the epilogue in L2
+          if constexpr (EPI) tma_load_2d_hint(slot + cc * (NC * 128), &p.tm_xc, &full[s], cc * 64, i * NC, l2_evict_first());
+          else tma_load_2d(slot + cc * (NC * 128), &p.tm_xc, &full[s], cc * 64, i * NC);
+        }
         ++n_issued;
         if (++s == L::kStages) { s = 0; ph ^= 1; }
       }
@@ -275,21 +279,28 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
         st_shared_v4(half + ((c16 ^ (lane & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
     };
-    auto store_tile = [&](const CUtensorMap* tm, uint32_t stg_off, int y0) {
+    auto store_tile = [&](const CUtensorMap* tm, uint32_t stg_off, int y0, bool stream = false) {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        for (int h = 0; h < D / 64; ++h) tma_store_2d(tm, s_stg + stg_off + h * L::kStgHalf, h * 64, y0);
+        if (stream) {  // written once and not read again here: leaves L2 first
+          const uint64_t pol = l2_evict_first();
+          for (int h = 0; h < D / 64; ++h) tma_store_2d_hint(tm, s_stg + stg_off + h * L::kStgHalf, h * 64, y0, pol);
+        } else {
+          for (int h = 0; h < D / 64; ++h) tma_store_2d(tm, s_stg + stg_off + h * L::kStgHalf, h * 64, y0);
+        }
         bulk_commit();
       }
     };
     // block epilogue: fetch the residual rows of this warp's 32-row output tile into its staging
     // buffer (same swizzled box as the store), add them, write the finished rows back in place
     uint32_t rph = 0;
-    auto load_residual = [&](const CUtensorMap* tm, uint32_t stg_off, int y0) {
+    auto load_residual = [&](const CUtensorMap* tm, uint32_t stg_off, int y0) {  // its last use: evict-first
       if (lane == 0) {
         mbar_arrive_expect_tx(&res_bar[ew], (uint32_t)(D * 32 * 2));
-        for (int h = 0; h < D / 64; ++h) tma_load_2d(s_stg + stg_off + h * L::kStgHalf, tm, &res_bar[ew], h * 64, y0);
+        const uint64_t pol = l2_evict_first();
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_2d_hint(s_stg + stg_off + h * L::kStgHalf, tm, &res_bar[ew], h * 64, y0, pol);
       }
     };
     auto drain_residual = [&]() {  // a wait failed with a residual load possibly in flight
@@ -554,8 +565,11 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
           if (res) {
             if (res_next != i) load_residual(&p.tm_res_c, stg_off, i * OC + 32 * quarter);
             // this group's tile after next: start its residual rows towards L2 now
-            if (lane == 0 && i + 2 * NG < cend)
-              for (int h = 0; h < D / 64; ++h) tma_prefetch_l2_2d(&p.tm_res_c, h * 64, (i + 2 * NG) * OC + 32 * quarter);
+            if (lane == 0 && i + 2 * NG < cend) {  // evict-last: it must survive until its load two tiles on
+              const uint64_t pol = l2_evict_last();
+              for (int h = 0; h < D / 64; ++h)
+                tma_prefetch_l2_2d_hint(&p.tm_res_c, h * 64, (i + 2 * NG) * OC + 32 * quarter, pol);
+            }
           }
           if (!mbar_wait(&acc_full[ab], (aphs >> ab) & 1, ctl, 312)) {
             if (res) drain_residual();
@@ -572,7 +586,7 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);
-          store_tile(&p.tm_yc, stg_off, i * OC + 32 * quarter);
+          store_tile(&p.tm_yc, stg_off, i * OC + 32 * quarter, true);
           // this group's next tile: its residual rows into the other staging buffer (whose last store,
           // two groups back, must have finished reading it)
           if (res && i + NG < cend) {

@@ -72,14 +72,17 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_proj_sm100_kernel(const __gr
       uint32_t s = 0, ph = 0;
       int n_issued = 0;
       bool ok = true;
+      // `in` streams past once (its 128-row block is shared only by the CTAs running the same m at the same
+      // time); the weight is read again by every wave of tiles, so it is kept in L2 ahead of `in`
+      const uint64_t pol_a = l2_evict_first(), pol_b = l2_evict_last();
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
         const int m0 = (t / nt) * BM, n0 = (t % nt) * BN;
         for (int kb = 0; kb < kb_n; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, ctl, 901)) { ok = false; break; }
           uint8_t* st = smem + s * kStage;
           mbar_arrive_expect_tx(&full[s], kStage);
-          tma_load_2d(st, &p.tm_a, &full[s], kb * BK, m0);
-          tma_load_2d(st + kA, &p.tm_b, &full[s], kb * BK, n0);
+          tma_load_2d_hint(st, &p.tm_a, &full[s], kb * BK, m0, pol_a);
+          tma_load_2d_hint(st + kA, &p.tm_b, &full[s], kb * BK, n0, pol_b);
           ++n_issued;
           if (++s == kStages) { s = 0; ph ^= 1; }
         }
