@@ -36,7 +36,7 @@ import rocs_inputs as ri  # noqa: E402
 from attention_ikbo_b200 import accounting as acc  # noqa: E402
 
 METRIC = "IKBO LCB/DCA TFLOP/s & candidates/s at 1 B200; % of bf16 tensor peak"
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 KERNEL_SRC = {"lcb": "attention_ikbo_b200/csrc/lcb_sm100.cu", "dca": "attention_ikbo_b200/csrc/dca_sm100.cu",
               "proj": "attention_ikbo_b200/csrc/proj_sm100.cu", "lcb_block": "attention_ikbo_b200/csrc/lcb_sm100.cu",
               "fm": "attention_ikbo_b200/csrc/fm_sm100.cu"}
@@ -663,7 +663,9 @@ def load_peaks():
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+        out = {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}
+        out["sm_max_mhz"] = float(d.get("sm_max_mhz", 1965.0))
+        return out, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
 
 
@@ -858,14 +860,33 @@ def timed_steps(parts, ikbo, torch, steps, flush, stream):
     return part_ms, launches
 
 
+# exp2 results per clock per SM of the MUFU (microbenchmarked on this B200: f32, f16x2 and bf16x2 alike)
+MUFU_EXP2_PER_CLK_SM = 16
+SM_COUNT = 148
+
+
+def exp_bound_tflops(dh, sm_max_mhz):
+    """Attention FLOP rate the exp2 unit allows: every score needs one exp2 and carries 4*dh FLOPs (QK^T and PV)."""
+    return MUFU_EXP2_PER_CLK_SM * SM_COUNT * sm_max_mhz * 1e6 * 4 * dh / 1e12
+
+
 def roofline_row(p, ms, peaks, peak_src):
     sec = ms * 1e-3
     if p.bound == "hbm":
         ach, peak, unit = p.bytes() / sec / 1e9, peaks["hbm_gbs"], "GB/s"
     else:
         ach, peak, unit = p.flops() / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    return {"kernel": p.name, "bound": p.bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
-            "traffic": ncu_traffic(p), "peak_source": f"{peak_src} (burst)"}
+    row = {"kernel": p.name, "bound": p.bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+           "traffic": ncu_traffic(p), "peak_source": f"{peak_src} (burst)"}
+    dh = getattr(getattr(p, "x", None), "dh", None)
+    if p.kernel == "dca" and dh is not None and exp_bound_tflops(dh, peaks["sm_max_mhz"]) < peak:
+        # dh = 64: the exponentials bound the attention below the tensor peak (MUFU throughput)
+        e = exp_bound_tflops(dh, peaks["sm_max_mhz"])
+        row.update({"bound": "alu", "peak": e, "frac": ach / e, "tensor_frac": ach / peak,
+                    "peak_source": f"exp2 rate: {MUFU_EXP2_PER_CLK_SM} per clock per SM (measured) x {SM_COUNT} SMs x "
+                                   f"{peaks['sm_max_mhz']:.0f} MHz x 4*dh FLOP per score; tensor_frac against the "
+                                   f"{peak_src} bf16 burst peak"})
+    return row
 
 
 # Workloads timed after the headline step and reported beside it (steps each; the explicit-expand
