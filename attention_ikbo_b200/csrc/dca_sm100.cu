@@ -101,6 +101,8 @@ struct Unit {
   int s0, L;       // first key row, number of keys
   int nkv;         // K/V tiles
   bool hasB;       // second 128-row tile has at least one valid row
+  int half;        // 0: whole unit; 1, 2: first / second half of a unit split along the keys
+  int slot;        // split units: index of the pair's merge area
 };
 
 __device__ __forceinline__ Unit load_unit(const DcaParams& p, int u) {
@@ -116,6 +118,19 @@ __device__ __forceinline__ Unit load_unit(const DcaParams& p, int u) {
   w.L = p.seq_off[w.r + 1] - w.s0;
   w.nkv = (w.L + BN - 1) / BN;
   w.hasB = w.row0 + BM < w.rows;
+  w.half = e.w & 3;
+  w.slot = e.w >> 2;
+  if (w.half) {  // a half of the keys: the first nkv/2 tiles, or the rest (the key range is rebased)
+    const int n0 = w.nkv / 2;
+    if (w.half == 1) {
+      w.L = n0 * BN;
+      w.nkv = n0;
+    } else {
+      w.s0 += n0 * BN;
+      w.L -= n0 * BN;
+      w.nkv -= n0;
+    }
+  }
   return w;
 }
 
@@ -556,6 +571,47 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       if (!mbar_wait(&o_full[x], ofph, ctl, 703)) { ok = false; break; }
       ofph ^= 1;
       tc_fence_after();
+      // A unit split along the keys: each half leaves its unnormalised O, running max and row sum in its merge
+      // area, then counts itself in; the half that counts second (it may run on either CTA, or on both the
+      // same) merges the two, O = (a O_own + b O_other) / (a l_own + b l_other), and writes the output.  No
+      // half waits for the other.
+      const float* oth = nullptr;  // the other half's O (second finisher only)
+      float a_own = 1.0f, b_oth = 0.0f;
+      if (w.half) {
+        const size_t area = (size_t)32 * (DH + 2);
+        float* mine = p.split_buf + ((((size_t)w.slot * 2 + (w.half - 1)) * 2 + x) * 4 + quarter) * area;
+#pragma unroll 1
+        for (int cc = 0; cc < DH / 32; ++cc) {  // [column/4][row][4]: each store a contiguous 512 bytes
+          uint32_t ov[32];
+          tmem_ld32(o_addr + cc * 32, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4)
+            *reinterpret_cast<uint4*>(mine + ((cc * 8 + k4) * 32 + lane) * 4) =
+                make_uint4(ov[4 * k4], ov[4 * k4 + 1], ov[4 * k4 + 2], ov[4 * k4 + 3]);
+        }
+        mine[DH * 32 + lane] = m_used;
+        mine[DH * 32 + 32 + lane] = l;
+        __threadfence();
+        __syncwarp();
+        int order = 0;
+        if (lane == 0) order = atomicAdd(&p.split_cnt[w.slot * 8 + x * 4 + quarter], 1);
+        order = __shfl_sync(0xffffffffu, order, 0);
+        if (order == 0) {  // the other half is still running: it writes this slab
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&o_empty[x]);
+          continue;
+        }
+        __threadfence();
+        oth = p.split_buf + ((((size_t)w.slot * 2 + (2 - w.half)) * 2 + x) * 4 + quarter) * area;
+        const float m_o = __ldcg(oth + DH * 32 + lane), l_o = __ldcg(oth + DH * 32 + 32 + lane);
+        const float mm = fmaxf(m_used, m_o);
+        a_own = ex2(m_used - mm);
+        b_oth = ex2(m_o - mm);
+        l = l * a_own + l_o * b_oth;
+        m_used = mm;
+      }
       const float inv = 1.0f / l;
       // This warp's 32 rows of the tile.  A full slab leaves through its shared-memory slab and a TMA store,
       // one 64-column box at a time: a handful of instructions per warp, where row-by-row 16-byte stores
@@ -570,6 +626,17 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         tmem_ld32(o_addr + cc * 64, ov[0]);
         tmem_ld32(o_addr + cc * 64 + 32, ov[1]);
         tmem_ld_wait_regs(ov[0], ov[1]);
+        if (oth) {  // second half of a split unit: a O_own + b O_other (the other's columns cc*64 .. +63)
+#pragma unroll
+          for (int k4 = 0; k4 < 16; ++k4) {
+            const float4 o4 = __ldcg(reinterpret_cast<const float4*>(oth + ((cc * 16 + k4) * 32 + lane) * 4));
+            uint32_t* v = &ov[k4 >> 3][(k4 & 7) * 4];
+            v[0] = __float_as_uint(__uint_as_float(v[0]) * a_own + o4.x * b_oth);
+            v[1] = __float_as_uint(__uint_as_float(v[1]) * a_own + o4.y * b_oth);
+            v[2] = __float_as_uint(__uint_as_float(v[2]) * a_own + o4.z * b_oth);
+            v[3] = __float_as_uint(__uint_as_float(v[3]) * a_own + o4.w * b_oth);
+          }
+        }
         if (tma_slab) {
           if (lane == 0) bulk_wait_read<0>();  // the slab's previous store has finished reading it
           __syncwarp();
@@ -619,7 +686,9 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
 
 // ------------------------------------------------------------------------------------
 // Work-unit table: one block.  units_r = H * ceil(q*N_r / 256); requests ordered by key
-// length descending (ties by index) so the longest units are claimed first.
+// length descending (ties by index) so the longest units are claimed first.  The last n_split units
+// in that order (the shortest) become two entries each, the halves of their K/V tiles, so that the
+// final partial wave of the persistent grid is made of half-length work.
 // Scratch (workspace): len[R], sorted[R], start[R+1].
 // ------------------------------------------------------------------------------------
 __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
@@ -664,6 +733,7 @@ __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
     __syncthreads();
   }
   int run = s_part[t] - sum;
+  const int whole = p.max_units - p.n_split, first_split = whole - p.n_split;
   for (int k = b0; k < b1; ++k) {
     const int r = sorted[k];
     const int rows = p.q * (p.cand_off[r + 1] - p.cand_off[r]);
@@ -672,12 +742,23 @@ __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
     for (int h = 0; h < p.H; ++h)
       for (int mb = 0; mb < nb; ++mb) {
         const int u = run + h * nb + mb;
-        if (u < p.max_units) p.units[u] = make_int4(r, h, mb * p.rows_per_unit, 0);
-        else record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 801);
+        int4 e = make_int4(r, h, mb * p.rows_per_unit, 0);
+        if (u >= whole || u < 0) {
+          record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 801);
+        } else if (u < first_split) {
+          p.units[u] = e;
+        } else {  // the two halves of split unit i, claimed one after the other
+          const int i = u - first_split;
+          e.w = (i << 2) | 1;
+          p.units[first_split + 2 * i] = e;
+          e.w = (i << 2) | 2;
+          p.units[first_split + 2 * i + 1] = e;
+        }
       }
     run += p.H * nb;
   }
-  if (t == T - 1 && s_part[T - 1] != p.max_units) record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 802);
+  if (t == T - 1 && s_part[T - 1] != whole) record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 802);
+  for (int i = t; i < 8 * p.n_split; i += T) p.split_cnt[i] = 0;
   if (t == 0) *p.ticket = 0;
 }
 

@@ -272,14 +272,35 @@ int64_t dca_units(const rocs_dca_args* a) {
   return n;
 }
 struct DcaLayout {
-  size_t scratch, units, body;
+  size_t scratch, units, split_cnt, split_buf, body;
 };
-DcaLayout dca_body(int64_t R, int64_t n_units) {
+// n_units: work-table entries (a split unit counts twice); n_split: units split in two along the keys
+DcaLayout dca_body(int64_t R, int64_t n_units, int64_t n_split = 0, int64_t dh = 128) {
   DcaLayout L;
   L.scratch = 0;
   L.units = a256((size_t)(3 * R + 1) * sizeof(int));
-  L.body = L.units + (size_t)n_units * sizeof(int4);
+  L.split_cnt = a256(L.units + (size_t)n_units * sizeof(int4));
+  L.split_buf = a256(L.split_cnt + (size_t)n_split * 8 * sizeof(int));
+  // per split unit: 2 halves x 2 tiles x 4 warps x 32 rows x (dh O values + max + sum), fp32
+  L.body = n_split ? L.split_buf + (size_t)n_split * 2 * 2 * 4 * 32 * (dh + 2) * sizeof(float) : L.units + (size_t)n_units * sizeof(int4);
   return L;
+}
+// Units split along the keys: the persistent grid claims units longest first, so with U units of equal
+// length on G CTAs the last U mod G of them form a partial wave of full-length units.  Those are split in
+// two, making the tail a wave of half-length work.  Only when every request with candidates has the same
+// number of K/V tiles, at least two (each half then has keys): with ragged key lengths the longest-first
+// claim order already evens out the tail, and splitting measured slower (merge and per-unit costs).
+int64_t dca_split_count(const rocs_dca_args* a, int64_t n_units) {
+  const int64_t G = sm_count();
+  if (n_units <= G || n_units % G == 0) return 0;
+  int64_t nkv = -1;
+  for (int64_t r = 0; r < a->R; ++r) {
+    if (a->cand_off_host[r + 1] == a->cand_off_host[r]) continue;
+    const int64_t t = (a->seq_off_host[r + 1] - a->seq_off_host[r] + 127) / 128;
+    if (t < 2 || (nkv >= 0 && t != nkv)) return 0;
+    nkv = t;
+  }
+  return n_units % G;
 }
 
 int dca_validate(const rocs_dca_args* a, int64_t* C, int64_t* T) {
@@ -307,8 +328,8 @@ int dca_validate(const rocs_dca_args* a, int64_t* C, int64_t* T) {
 // ticket: the work counter of this launch (default: the header's); two launches that run at the same
 // time on one header use different counters
 int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHeader* hdr, uint8_t* w,
-            cudaStream_t st, int* launches, bool reset_header = true, int* ticket = nullptr) {
-  const DcaLayout L = dca_body(a->R, n_units);
+            cudaStream_t st, int* launches, bool reset_header = true, int* ticket = nullptr, int64_t n_split = 0) {
+  const DcaLayout L = dca_body(a->R, n_units + n_split, n_split, a->dh);
   if (n_units >= (int64_t(1) << 31)) return ROCS_ERR_UNSUPPORTED;
   if (reset_header && cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return ROCS_ERR_CUDA;
   if (n_units == 0) return ROCS_OK;
@@ -323,7 +344,9 @@ int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHea
   sp.q = (int)a->q;
   sp.H = (int)a->H;
   sp.rows_per_unit = dca_rows_per_unit();
-  sp.max_units = (int)n_units;
+  sp.max_units = (int)(n_units + n_split);
+  sp.n_split = (int)n_split;
+  sp.split_cnt = reinterpret_cast<int*>(w + L.split_cnt);
   if (launch_dca_schedule(sp, st) != cudaSuccess) return ROCS_ERR_CUDA;
   DcaParams p;
   std::memset(&p, 0, sizeof(p));
@@ -341,6 +364,8 @@ int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHea
   p.cand_off = a->cand_off_dev;
   p.seq_off = a->seq_off_dev;
   p.units = sp.units;
+  p.split_cnt = sp.split_cnt;
+  p.split_buf = reinterpret_cast<float*>(w + L.split_buf);
   p.o = static_cast<__nv_bfloat16*>(a->o_ptr);
   p.lse = a->lse_ptr;
   p.ws = sp.ws;
@@ -348,10 +373,10 @@ int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHea
   p.R = (int)a->R;
   p.q = (int)a->q;
   p.H = (int)a->H;
-  p.n_units = (int)n_units;
+  p.n_units = (int)(n_units + n_split);
   p.scale_log2 = a->scale * 1.4426950408889634f;
   p.wait_limit_ns = kDefaultWaitLimitNs;
-  int64_t grid = n_units < sm_count() ? n_units : sm_count();
+  int64_t grid = n_units + n_split < sm_count() ? n_units + n_split : sm_count();
   if (launch_dca_sm100(p, (int)a->dh, (int)grid, st) != cudaSuccess) return ROCS_ERR_CUDA;
   *launches = 2;
   return ROCS_OK;
@@ -443,21 +468,23 @@ int rocs_lcb_block_forward(const rocs_lcb_args* a, const rocs_lcb_epilogue* epi_
 size_t rocs_dca_workspace_size(const rocs_dca_args* a) {
   int64_t C, T;
   if (dca_validate(a, &C, &T) != ROCS_OK) return 0;
-  return sizeof(WsHeader) + dca_body(a->R, dca_units(a)).body;
+  const int64_t n_units = dca_units(a), n_split = dca_split_count(a, n_units);
+  return sizeof(WsHeader) + dca_body(a->R, n_units + n_split, n_split, a->dh).body;
 }
 
 int rocs_dca_forward(const rocs_dca_args* a, rocs_stream_t stream) {
   int64_t C = 0, T = 0;
   int rc = dca_validate(a, &C, &T);
   if (rc) return rc;
-  const int64_t n_units = dca_units(a);
-  if (!a->workspace || a->workspace_bytes < sizeof(WsHeader) + dca_body(a->R, n_units).body ||
+  const int64_t n_units = dca_units(a), n_split = dca_split_count(a, n_units);
+  if (!a->workspace ||
+      a->workspace_bytes < sizeof(WsHeader) + dca_body(a->R, n_units + n_split, n_split, a->dh).body ||
       (reinterpret_cast<uintptr_t>(a->workspace) & 255))
     return ROCS_ERR_WORKSPACE;
   int launches = 0;
   WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
   rc = dca_run(a, C, T, n_units, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream),
-               &launches);
+               &launches, true, nullptr, n_split);
   if (rc == ROCS_OK) g_last_launches = launches;
   return rc;
 }

@@ -125,6 +125,21 @@ def test_dca_long_full_size_sampled(ikbo, oracle_mod):
     check(oracle_mod, x, o, lse, sel=sel)
 
 
+@pytest.mark.parametrize("dh", [64, 128])
+def test_dca_split_tail_units(ikbo, oracle_mod, dh):
+    """More work units than the GPU has SMs and every request with the same number (>= 2) of K/V tiles: the
+    last (units mod SMs) units in claim order are split in two along the keys, each half leaves its partial
+    result and the half that finishes second merges them.  Every candidate against the oracle."""
+    counts = ri.uniform_int(91, 1, 1, 300, 80)
+    lengths = ri.uniform_int(92, 2, 641, 768, 80)  # six K/V tiles each, ragged within the last tile
+    x = ri.make_dca("split", counts, lengths, 1, 2, dh, 93)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    units = x.H * sum((x.q * int(n) + 255) // 256 for n in counts)
+    assert units > sms and units % sms  # the premise: a partial last wave, so some units are split
+    o, lse = run_dca(ikbo, x)
+    check(oracle_mod, x, o, lse)
+
+
 def _f32_to_bf16(a):
     """Round-to-nearest-even fp32 -> bf16 bits (finite inputs)."""
     u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
