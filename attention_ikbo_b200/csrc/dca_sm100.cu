@@ -53,12 +53,15 @@ constexpr int kRowsPerUnit = 2 * BM;
 
 template <int DH>
 struct DcaSmem {
-  static constexpr uint32_t kTile = BM * DH * 2;  // one Q tile or one K/V tile (bf16)
-  static constexpr int kRing = DH == 128 ? 4 : 10;
+  static constexpr uint32_t kTile = BM * DH * 2;  // one Q tile or one K/V tile of one head (bf16)
+  // K/V ring slot: one head's tile (dh = 128), or room for two heads' tiles (dh = 64: a head pair's)
+  static constexpr int kHeadsPerSlot = DH == 128 ? 1 : 2;  // head pairs are formed at dh = 64 only
+  static constexpr uint32_t kSlot = kHeadsPerSlot * kTile;
+  static constexpr int kRing = DH == 128 ? 4 : 5;
   static constexpr uint32_t kStage = 32 * 128;     // per softmax warp: 32 rows x 64 columns of O (bf16)
   static constexpr uint32_t off_q = 0;
   static constexpr uint32_t off_ring = 2 * kTile;
-  static constexpr uint32_t off_stage = off_ring + kRing * kTile;  // 8 warps x kStage, 1024-byte aligned
+  static constexpr uint32_t off_stage = off_ring + kRing * kSlot;  // 8 warps x kStage, 1024-byte aligned
   static constexpr uint32_t off_bar = off_stage + 8 * kStage;
   static constexpr uint32_t n_bars = 2 * kRing + 2 * 8 + 1 + 4;
   static constexpr uint32_t off_misc = off_bar + n_bars * 8;
@@ -103,6 +106,8 @@ struct Unit {
   bool hasB;       // second 128-row tile has at least one valid row
   int half;        // 0: whole unit; 1, 2: first / second half of a unit split along the keys
   int slot;        // split units: index of the pair's merge area
+  int nh;          // heads whose K/V the unit reads: 2 for a head pair (tile B = the next head, same rows)
+  int hB, rowB0;   // head and first row (within the request's rows) of tile B
 };
 
 __device__ __forceinline__ Unit load_unit(const DcaParams& p, int u) {
@@ -117,9 +122,13 @@ __device__ __forceinline__ Unit load_unit(const DcaParams& p, int u) {
   w.s0 = p.seq_off[w.r];
   w.L = p.seq_off[w.r + 1] - w.s0;
   w.nkv = (w.L + BN - 1) / BN;
-  w.hasB = w.row0 + BM < w.rows;
+  const bool paired = (e.w >> 2) & 1;
+  w.nh = paired ? 2 : 1;
+  w.hB = paired ? w.h + 1 : w.h;
+  w.rowB0 = paired ? w.row0 : w.row0 + BM;
+  w.hasB = paired || w.row0 + BM < w.rows;
   w.half = e.w & 3;
-  w.slot = e.w >> 2;
+  w.slot = e.w >> 3;
   if (w.half) {  // a half of the keys: the first nkv/2 tiles, or the rest (the key range is rebased)
     const int n0 = w.nkv / 2;
     if (w.half == 1) {
@@ -216,12 +225,15 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       uint32_t rs = 0, rph = 0, ws_ = 0, wph = 0, qeph[2] = {0, 0};
       int n_issued = 0;
       bool ok = true;
-      auto load_kv = [&](const CUtensorMap* tm, int y, int x0) -> bool {
+      // one K/V tile (128 keys) of heads h0 .. h0+nh-1 into the next ring slot, head hh at offset hh * kTile
+      auto load_kv = [&](const CUtensorMap* tm, int y, int h0, int nh) -> bool {
         if (!mbar_wait(&ring_empty[rs], rph ^ 1, ctl, 501)) return false;
-        uint8_t* slot = s_ring + rs * L::kTile;
-        mbar_arrive_expect_tx(&ring_full[rs], L::kTile);
+        uint8_t* slot = s_ring + rs * L::kSlot;
+        mbar_arrive_expect_tx(&ring_full[rs], nh * L::kTile);
+        for (int hh = 0; hh < nh; ++hh)
 #pragma unroll
-        for (int cc = 0; cc < DH / 64; ++cc) tma_load_2d(slot + cc * (BM * 128), tm, &ring_full[rs], x0 + cc * 64, y);
+          for (int cc = 0; cc < DH / 64; ++cc)
+            tma_load_2d(slot + hh * L::kTile + cc * (BM * 128), tm, &ring_full[rs], (h0 + hh) * DH + cc * 64, y);
         ++n_issued;
         if (++rs == kRing) { rs = 0; rph ^= 1; }
         return true;
@@ -239,24 +251,28 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         if (item < 0) break;
         const Unit w = load_unit(p, item);
         if (w.nkv == 0) continue;
-        const int x0 = w.h * DH;
         for (int x = 0; x < (w.hasB ? 2 : 1); ++x) {
           if (!mbar_wait(&q_empty[x], qeph[x] ^ 1, ctl, 503)) { ok = false; break; }
           qeph[x] ^= 1;
           mbar_arrive_expect_tx(&q_full[x], L::kTile);
 #pragma unroll
           for (int cc = 0; cc < DH / 64; ++cc)
-            tma_load_2d(s_q + x * L::kTile + cc * (BM * 128), &p.tm_q, &q_full[x], x0 + cc * 64,
-                        w.qbase + w.row0 + x * BM);
+            tma_load_2d(s_q + x * L::kTile + cc * (BM * 128), &p.tm_q, &q_full[x],
+                        ((L::kHeadsPerSlot == 2 && x) ? w.hB : w.h) * DH + cc * 64,
+                        w.qbase + ((L::kHeadsPerSlot == 2) ? (x ? w.rowB0 : w.row0) : w.row0 + x * BM));
         }
         if (!ok) break;
-        // K/V in the order the MMA issuer consumes them: K0, (K1, V0), (K2, V1), ..., V_last
-        ok = load_kv(&p.tm_k, w.s0, x0);
+        // K/V in the order the MMA issuer consumes them: K0, (K1, V0), (K2, V1), ..., V_last; a head pair
+        // loads each tile for both heads into one slot
+        auto kv_step = [&](const CUtensorMap* tm, int y) -> bool {
+          return load_kv(tm, y, w.h, L::kHeadsPerSlot == 2 ? w.nh : 1);
+        };
+        ok = kv_step(&p.tm_k, w.s0);
         for (int j = 1; ok && j < w.nkv; ++j) {
-          ok = load_kv(&p.tm_k, w.s0 + j * BN, x0);
-          if (ok) ok = load_kv(&p.tm_v, w.s0 + (j - 1) * BN, x0);
+          ok = kv_step(&p.tm_k, w.s0 + j * BN);
+          if (ok) ok = kv_step(&p.tm_v, w.s0 + (j - 1) * BN);
         }
-        if (ok) ok = load_kv(&p.tm_v, w.s0 + (w.nkv - 1) * BN, x0);
+        if (ok) ok = kv_step(&p.tm_v, w.s0 + (w.nkv - 1) * BN);
       }
       if (!ok) {
         for (int k = n_issued > kRing ? n_issued - kRing : 0; k < n_issued; ++k)
@@ -274,11 +290,11 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       const uint32_t q0 = smem_u32(s_q);
       auto next_slot = [&](uint32_t& slot_addr, int where) -> bool {
         if (!mbar_wait(&ring_full[rs], rph, ctl, where)) return false;
-        slot_addr = smem_u32(s_ring + rs * L::kTile);
+        slot_addr = smem_u32(s_ring + rs * L::kSlot);
         return true;
       };
       auto release_slot = [&](uint32_t slot_addr) {  // slots are consumed in ring order
-        const uint32_t idx = (slot_addr - smem_u32(s_ring)) / L::kTile;
+        const uint32_t idx = (slot_addr - smem_u32(s_ring)) / L::kSlot;
         umma_commit(&ring_empty[idx]);
       };
       auto advance = [&]() {
@@ -337,26 +353,28 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         }
         if (!ok) break;
         tc_fence_after();
+        // a head pair's two tiles read the two halves of each K/V slot (tile B at byte offset pb)
+        const uint32_t pb = (L::kHeadsPerSlot == 2 && w.nh == 2) ? L::kTile : 0u;
         uint32_t kslot, vslot;
         if (!next_slot(kslot, 605)) { ok = false; break; }
         advance();
         tc_fence_after();
         if constexpr (kSepP) {
-          for (int x = 0; x < nx && ok; ++x) ok = issue_s_free(x, kslot);
+          for (int x = 0; x < nx && ok; ++x) ok = issue_s_free(x, kslot + pb * x);
           if (!ok) break;
           release_slot(kslot);
           // per K/V step: S of the next tile as soon as the softmax has read the current one, then P V
           for (int j = 1; j < w.nkv; ++j) {
             if (!next_slot(kslot, 606)) { ok = false; break; }
             advance();
-            for (int x = 0; x < nx && ok; ++x) ok = issue_s_free(x, kslot);
+            for (int x = 0; x < nx && ok; ++x) ok = issue_s_free(x, kslot + pb * x);
             if (!ok) break;
             release_slot(kslot);
             if (!next_slot(vslot, 607)) { ok = false; break; }
             advance();
             for (int x = 0; x < nx; ++x) {
               if (!wait_p(x, j == 1)) { ok = false; break; }
-              issue_pv(x, vslot, j > 1);
+              issue_pv(x, vslot + pb * x, j > 1);
               umma_commit(&pv_done[x]);
             }
             if (!ok) break;
@@ -368,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
           advance();
           for (int x = 0; x < nx; ++x) {
             if (!wait_p(x, w.nkv == 1)) { ok = false; break; }
-            issue_pv(x, vslot, w.nkv > 1);
+            issue_pv(x, vslot + pb * x, w.nkv > 1);
             umma_commit(&pv_done[x]);
             umma_commit(&o_full[x]);
           }
@@ -377,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
           continue;
         }
         issue_s(0, kslot);
-        if (nx == 2) issue_s(1, kslot);
+        if (nx == 2) issue_s(1, kslot + pb);
         release_slot(kslot);
         for (int j = 1; j < w.nkv; ++j) {
           if (!next_slot(kslot, 606)) { ok = false; break; }
@@ -386,8 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
           advance();
           for (int x = 0; x < nx; ++x) {
             if (!wait_p(x, j == 1)) { ok = false; break; }
-            issue_pv(x, vslot, j > 1);
-            issue_s(x, kslot);
+            issue_pv(x, vslot + pb * x, j > 1);
+            issue_s(x, kslot + pb * x);
           }
           if (!ok) break;
           release_slot(vslot);
@@ -399,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
         advance();
         for (int x = 0; x < nx; ++x) {
           if (!wait_p(x, w.nkv == 1)) { ok = false; break; }
-          issue_pv(x, vslot, w.nkv > 1);
+          issue_pv(x, vslot + pb * x, w.nkv > 1);
           umma_commit(&o_full[x]);
         }
         if (!ok) break;
@@ -432,14 +450,16 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       if (item < 0) break;
       const Unit w = load_unit(p, item);
       if (x == 1 && !w.hasB) continue;
-      const int row = w.row0 + x * BM + 32 * quarter + (int)lane;  // row within the request
+      const int hx = (L::kHeadsPerSlot == 2 && x) ? w.hB : w.h;          // this tile's head
+      const int tile0 = (L::kHeadsPerSlot == 2) ? (x ? w.rowB0 : w.row0) : w.row0 + x * BM;  // its first row
+      const int row = tile0 + 32 * quarter + (int)lane;  // row within the request
       const bool row_ok = row < w.rows;
-      __nv_bfloat16* orow = p.o + ((size_t)(w.qbase + row) * p.H + w.h) * DH;
+      __nv_bfloat16* orow = p.o + ((size_t)(w.qbase + row) * p.H + hx) * DH;
       if (w.nkv == 0) {  // request without keys: O = 0, LSE = -inf
         if (row_ok) {
 #pragma unroll
           for (int k = 0; k < DH / 8; ++k) st_global_v4(orow + 8 * k, 0u, 0u, 0u, 0u);
-          if (p.lse) p.lse[(size_t)(w.qbase + row) * p.H + w.h] = -INFINITY;
+          if (p.lse) p.lse[(size_t)(w.qbase + row) * p.H + hx] = -INFINITY;
         }
         continue;
       }
@@ -618,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       // (32 rows apart per instruction) would queue thousands of small writes in the SM's memory pipeline, in
       // front of the producer's and the issuer's own memory instructions.  A slab cut by the end of the
       // request's rows is stored row by row, so that no row of the next request is written.
-      const int slab0 = w.row0 + x * BM + 32 * quarter;  // first row of the slab within the request
+      const int slab0 = tile0 + 32 * quarter;  // first row of the slab within the request
       const bool tma_slab = slab0 + 32 <= w.rows;
 #pragma unroll 1
       for (int cc = 0; cc < DH / 64; ++cc) {
@@ -652,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&p.tm_o, stage, w.h * DH + cc * 64, w.qbase + slab0);
+            tma_store_2d(&p.tm_o, stage, hx * DH + cc * 64, w.qbase + slab0);
             bulk_commit();
           }
         } else if (row_ok) {
@@ -669,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_empty[x]);
-      if (row_ok && p.lse) p.lse[(size_t)(w.qbase + row) * p.H + w.h] = (m_used + lg2(l)) * 0.69314718055994531f;
+      if (row_ok && p.lse) p.lse[(size_t)(w.qbase + row) * p.H + hx] = (m_used + lg2(l)) * 0.69314718055994531f;
     }
     (void)ok;
     if (lane == 0) bulk_wait<0>();  // every TMA store of this warp has completed
@@ -715,14 +735,22 @@ __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
     sorted[rank] = r;
   }
   __syncthreads();
-  // units of each sorted position, exclusive scan over positions
+  // units of each sorted position, exclusive scan over positions.  With pair_heads, a request's last chunk of
+  // at most 128 rows (one query tile) is taken for two heads at once: one unit per head pair, tile B holding
+  // the next head's rows (an odd last head stays alone).
   const int per = (R + T - 1) / T;
   const int b0 = min(R, t * per), b1 = min(R, b0 + per);
+  auto units_of = [&](int rows, int& nb, bool& pair_last) {
+    nb = (rows + p.rows_per_unit - 1) / p.rows_per_unit;
+    pair_last = p.pair_heads && p.H >= 2 && nb > 0 && rows - (nb - 1) * p.rows_per_unit <= BM;
+    return pair_last ? p.H * (nb - 1) + (p.H + 1) / 2 : p.H * nb;
+  };
   int sum = 0;
   for (int k = b0; k < b1; ++k) {
     const int r = sorted[k];
-    const int rows = p.q * (p.cand_off[r + 1] - p.cand_off[r]);
-    sum += p.H * ((rows + p.rows_per_unit - 1) / p.rows_per_unit);
+    int nb;
+    bool pl;
+    sum += units_of(p.q * (p.cand_off[r + 1] - p.cand_off[r]), nb, pl);
   }
   s_part[t] = sum;
   __syncthreads();
@@ -734,28 +762,32 @@ __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
   }
   int run = s_part[t] - sum;
   const int whole = p.max_units - p.n_split, first_split = whole - p.n_split;
+  auto put = [&](int u, int4 e) {
+    if (u >= whole || u < 0) {
+      record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 801);
+    } else if (u < first_split) {
+      p.units[u] = e;
+    } else {  // the two halves of split unit i, claimed one after the other
+      const int i = u - first_split;
+      e.w |= (i << 3) | 1;
+      p.units[first_split + 2 * i] = e;
+      e.w ^= 3;  // half 1 -> 2
+      p.units[first_split + 2 * i + 1] = e;
+    }
+  };
   for (int k = b0; k < b1; ++k) {
     const int r = sorted[k];
-    const int rows = p.q * (p.cand_off[r + 1] - p.cand_off[r]);
-    const int nb = (rows + p.rows_per_unit - 1) / p.rows_per_unit;
+    int nb;
+    bool pl;
+    const int n = units_of(p.q * (p.cand_off[r + 1] - p.cand_off[r]), nb, pl);
     start[k] = run;
+    const int nbw = pl ? nb - 1 : nb;  // chunks taken one head at a time
     for (int h = 0; h < p.H; ++h)
-      for (int mb = 0; mb < nb; ++mb) {
-        const int u = run + h * nb + mb;
-        int4 e = make_int4(r, h, mb * p.rows_per_unit, 0);
-        if (u >= whole || u < 0) {
-          record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 801);
-        } else if (u < first_split) {
-          p.units[u] = e;
-        } else {  // the two halves of split unit i, claimed one after the other
-          const int i = u - first_split;
-          e.w = (i << 2) | 1;
-          p.units[first_split + 2 * i] = e;
-          e.w = (i << 2) | 2;
-          p.units[first_split + 2 * i + 1] = e;
-        }
-      }
-    run += p.H * nb;
+      for (int mb = 0; mb < nbw; ++mb) put(run + h * nbw + mb, make_int4(r, h, mb * p.rows_per_unit, 0));
+    if (pl)
+      for (int hp = 0; 2 * hp < p.H; ++hp)
+        put(run + p.H * nbw + hp, make_int4(r, 2 * hp, nbw * p.rows_per_unit, 2 * hp + 1 < p.H ? 4 : 0));
+    run += n;
   }
   if (t == T - 1 && s_part[T - 1] != whole) record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 802);
   for (int i = t; i < 8 * p.n_split; i += T) p.split_cnt[i] = 0;

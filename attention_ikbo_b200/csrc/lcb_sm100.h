@@ -48,7 +48,7 @@ struct DcaParams {
   CUtensorMap tm_o;  // O viewed as [C*q, H*dh], box {64, 32}   (stores)
   const int32_t* cand_off;
   const int32_t* seq_off;
-  const int4* units;  // work-unit table {r, h, row0, split}: split 0 = whole unit, else (slot << 2) | half (1, 2)
+  const int4* units;  // work-unit table {r, h, row0, w}: w = (split slot << 3) | (head pair << 2) | half (0 whole, 1, 2)
   int* ticket;        // work-unit counter (zeroed by the schedule kernel)
   float* split_buf;   // split units: per slot, half, tile, warp: unnormalised O [dh/4][32][4], m [32], l [32]
   int* split_cnt;     // split units: per slot, tile and warp, halves finished (zeroed by the schedule kernel)
@@ -71,6 +71,7 @@ struct DcaSchedParams {
   int* split_cnt;  // [n_split * 8], zeroed here
   int R, q, H, rows_per_unit, max_units;
   int n_split;     // the last n_split units in claim order are split in two along the keys
+  int pair_heads;  // a request's last chunk of <= 128 rows is one unit per head pair
 };
 cudaError_t launch_dca_schedule(const DcaSchedParams& p, cudaStream_t st);
 

@@ -262,15 +262,23 @@ int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaSt
 
 // ---------------------------------------------------------------- DCA
 // workspace = [WsHeader][body]; body = [scratch: 3R+1 ints][work units: n_units int4]
-int64_t dca_units(const rocs_dca_args* a) {
+// Work units: per request and head, chunks of 256 query rows (two 128-row tiles).  pair_heads: a request's last
+// chunk of at most 128 rows is one unit for two heads (tile B = the next head), as the schedule kernel builds it.
+int64_t dca_units(const rocs_dca_args* a, bool pair_heads = false) {
   const int rpu = dca_rows_per_unit();
   int64_t n = 0;
   for (int64_t r = 0; r < a->R; ++r) {
     const int64_t rows = a->q * (int64_t)(a->cand_off_host[r + 1] - a->cand_off_host[r]);
-    n += a->H * ((rows + rpu - 1) / rpu);
+    const int64_t nb = (rows + rpu - 1) / rpu;
+    if (pair_heads && a->H >= 2 && nb > 0 && rows - (nb - 1) * rpu <= rpu / 2)
+      n += a->H * (nb - 1) + (a->H + 1) / 2;
+    else
+      n += a->H * nb;
   }
   return n;
 }
+// Head pairs are formed where both heads' K/V tiles fit the ring: dh = 64
+bool dca_pair_heads(const rocs_dca_args* a) { return a->dh == 64; }
 struct DcaLayout {
   size_t scratch, units, split_cnt, split_buf, body;
 };
@@ -328,7 +336,8 @@ int dca_validate(const rocs_dca_args* a, int64_t* C, int64_t* T) {
 // ticket: the work counter of this launch (default: the header's); two launches that run at the same
 // time on one header use different counters
 int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHeader* hdr, uint8_t* w,
-            cudaStream_t st, int* launches, bool reset_header = true, int* ticket = nullptr, int64_t n_split = 0) {
+            cudaStream_t st, int* launches, bool reset_header = true, int* ticket = nullptr, int64_t n_split = 0,
+            bool pair_heads = false) {
   const DcaLayout L = dca_body(a->R, n_units + n_split, n_split, a->dh);
   if (n_units >= (int64_t(1) << 31)) return ROCS_ERR_UNSUPPORTED;
   if (reset_header && cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st) != cudaSuccess) return ROCS_ERR_CUDA;
@@ -346,6 +355,7 @@ int dca_run(const rocs_dca_args* a, int64_t C, int64_t T, int64_t n_units, WsHea
   sp.rows_per_unit = dca_rows_per_unit();
   sp.max_units = (int)(n_units + n_split);
   sp.n_split = (int)n_split;
+  sp.pair_heads = pair_heads ? 1 : 0;
   sp.split_cnt = reinterpret_cast<int*>(w + L.split_cnt);
   if (launch_dca_schedule(sp, st) != cudaSuccess) return ROCS_ERR_CUDA;
   DcaParams p;
@@ -468,7 +478,7 @@ int rocs_lcb_block_forward(const rocs_lcb_args* a, const rocs_lcb_epilogue* epi_
 size_t rocs_dca_workspace_size(const rocs_dca_args* a) {
   int64_t C, T;
   if (dca_validate(a, &C, &T) != ROCS_OK) return 0;
-  const int64_t n_units = dca_units(a), n_split = dca_split_count(a, n_units);
+  const int64_t n_units = dca_units(a, dca_pair_heads(a)), n_split = dca_split_count(a, n_units);
   return sizeof(WsHeader) + dca_body(a->R, n_units + n_split, n_split, a->dh).body;
 }
 
@@ -476,7 +486,8 @@ int rocs_dca_forward(const rocs_dca_args* a, rocs_stream_t stream) {
   int64_t C = 0, T = 0;
   int rc = dca_validate(a, &C, &T);
   if (rc) return rc;
-  const int64_t n_units = dca_units(a), n_split = dca_split_count(a, n_units);
+  const bool pair = dca_pair_heads(a);
+  const int64_t n_units = dca_units(a, pair), n_split = dca_split_count(a, n_units);
   if (!a->workspace ||
       a->workspace_bytes < sizeof(WsHeader) + dca_body(a->R, n_units + n_split, n_split, a->dh).body ||
       (reinterpret_cast<uintptr_t>(a->workspace) & 255))
@@ -484,7 +495,7 @@ int rocs_dca_forward(const rocs_dca_args* a, rocs_stream_t stream) {
   int launches = 0;
   WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
   rc = dca_run(a, C, T, n_units, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream),
-               &launches, true, nullptr, n_split);
+               &launches, true, nullptr, n_split, pair);
   if (rc == ROCS_OK) g_last_launches = launches;
   return rc;
 }

@@ -140,6 +140,16 @@ def test_dca_split_tail_units(ikbo, oracle_mod, dh):
     check(oracle_mod, x, o, lse)
 
 
+def test_dca_head_pairs(ikbo, oracle_mod):
+    """dh = 64: a request's last chunk of at most 128 query rows is one unit for two heads (tile B holds the
+    next head's rows); with H = 5 the last head of each such chunk stays alone.  Requests whose rows end in
+    a short chunk, one whose rows fill whole chunks, an empty one and ragged keys; every candidate against
+    the oracle."""
+    x = ri.make_dca("pairs", [3, 64, 0, 129, 256, 190, 1], [300, 129, 50, 700, 1, 255, 1000], 2, 5, 64, 97)
+    o, lse = run_dca(ikbo, x)
+    check(oracle_mod, x, o, lse)
+
+
 def _f32_to_bf16(a):
     """Round-to-nearest-even fp32 -> bf16 bits (finite inputs)."""
     u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
