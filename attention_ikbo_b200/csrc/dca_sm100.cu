@@ -709,7 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
 // length descending (ties by index) so the longest units are claimed first.  The last n_split units
 // in that order (the shortest) become two entries each, the halves of their K/V tiles, so that the
 // final partial wave of the persistent grid is made of half-length work.
-// Scratch (workspace): len[R], sorted[R], start[R+1].
+// Scratch (workspace): len[R], sorted[R], start[R+1] (first unit of each sorted position, then the total).
 // ------------------------------------------------------------------------------------
 __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
   // the attention kernel may start its prologue now; it waits for this grid before claiming units
@@ -775,21 +775,40 @@ __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
       p.units[first_split + 2 * i + 1] = e;
     }
   };
-  for (int k = b0; k < b1; ++k) {
+  for (int k = b0; k < b1; ++k) {  // first unit of each sorted position
     const int r = sorted[k];
     int nb;
     bool pl;
-    const int n = units_of(p.q * (p.cand_off[r + 1] - p.cand_off[r]), nb, pl);
     start[k] = run;
-    const int nbw = pl ? nb - 1 : nb;  // chunks taken one head at a time
-    for (int h = 0; h < p.H; ++h)
-      for (int mb = 0; mb < nbw; ++mb) put(run + h * nbw + mb, make_int4(r, h, mb * p.rows_per_unit, 0));
-    if (pl)
-      for (int hp = 0; 2 * hp < p.H; ++hp)
-        put(run + p.H * nbw + hp, make_int4(r, 2 * hp, nbw * p.rows_per_unit, 2 * hp + 1 < p.H ? 4 : 0));
-    run += n;
+    run += units_of(p.q * (p.cand_off[r + 1] - p.cand_off[r]), nb, pl);
   }
-  if (t == T - 1 && s_part[T - 1] != whole) record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 802);
+  if (t == T - 1) {
+    start[R] = s_part[T - 1];
+    if (s_part[T - 1] != whole) record_error(p.ws, ROCS_ERR_DEVICE_INDEX, 802);
+  }
+  __syncthreads();
+  // every thread writes every T-th unit: its sorted position by binary search over start[], then the unit's
+  // head and chunk (a few requests can own most of the units, so positions are not split over threads)
+  const int n_all = start[R] < whole ? start[R] : whole;
+  for (int u = t; u < n_all; u += T) {
+    int lo = 0, hi = R - 1;  // last k with start[k] <= u
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (start[mid] <= u) lo = mid;
+      else hi = mid - 1;
+    }
+    const int r = sorted[lo], local = u - start[lo];
+    int nb;
+    bool pl;
+    units_of(p.q * (p.cand_off[r + 1] - p.cand_off[r]), nb, pl);
+    const int nbw = pl ? nb - 1 : nb;  // chunks taken one head at a time
+    if (local < p.H * nbw)
+      put(u, make_int4(r, local / nbw, (local % nbw) * p.rows_per_unit, 0));
+    else {
+      const int hp = local - p.H * nbw;
+      put(u, make_int4(r, 2 * hp, nbw * p.rows_per_unit, 2 * hp + 1 < p.H ? 4 : 0));
+    }
+  }
   for (int i = t; i < 8 * p.n_split; i += T) p.split_cnt[i] = 0;
   if (t == 0) *p.ticket = 0;
 }
