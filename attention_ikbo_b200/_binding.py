@@ -2,6 +2,7 @@
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import numpy as np
@@ -146,6 +147,23 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _on_tensor_device(fn):
+    """Run ``fn`` with the device of its first CUDA tensor argument current (else the ``device``
+    keyword's, else the current device), so that the library's per-device state (SM count, kernel
+    attributes, the no-alloc scratch array) and the default stream belong to the device the data is on."""
+    @functools.wraps(fn)
+    def run(*args, **kw):
+        for t in list(args) + list(kw.values()):
+            if isinstance(t, torch.Tensor) and t.is_cuda:
+                with torch.cuda.device(t.device):
+                    return fn(*args, **kw)
+        if kw.get("device") is not None and torch.device(kw["device"]).index is not None:
+            with torch.cuda.device(torch.device(kw["device"])):
+                return fn(*args, **kw)
+        return fn(*args, **kw)
+    return run
+
+
 def offsets(off, device="cuda"):
     """CSR offsets as the pair the C ABI needs: (device int32 tensor, host int32 numpy array).
 
@@ -203,6 +221,7 @@ def _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req, y_cand):
     return a, (off_d, off_h), y_req, y_cand
 
 
+@_on_tensor_device
 def rocs_lcb_forward(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req=None, y_cand=None, workspace=None,
                      stream=None, expand=False):
     """IKBO-LCB.  Returns ``(y_req [R,o_r,d], y_cand [C,o_c,d])``; see ``rocs_lcb_forward`` in the header.
@@ -253,6 +272,7 @@ def rocs_lcb_noalloc_read_status(device=None, stream=None):
     return code.value, detail.value
 
 
+@_on_tensor_device
 def rocs_lcb_forward_fault_injection(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, skip_release_request,
                                      wait_limit_ns, stream=None):
     """Test hook: LCB whose request ``skip_release_request`` never signals its Z; the kernel must end
@@ -289,6 +309,7 @@ def _epilogue(e, y_shape, dev, keep):
                        act=ACTS[act] if isinstance(act, str) else int(act))
 
 
+@_on_tensor_device
 def rocs_lcb_block_forward(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, epi_req=None, epi_cand=None, y_req=None,
                            y_cand=None, workspace=None, stream=None):
     """LCB block: IKBO-LCB with each group's bias / residual / norm / activation fused into the epilogue.
@@ -338,6 +359,7 @@ def _dca_args(q_t, k_t, v_t, cand_off, seq_off, q_tokens, scale, o, lse):
     return a, (co_d, co_h, so_d, so_h), o, lse
 
 
+@_on_tensor_device
 def rocs_dca_forward(q_t, k_t, v_t, cand_off, seq_off, q_tokens, scale, o=None, lse=True, workspace=None,
                      stream=None, expand_chunk=None):
     """IKBO-DCA.  Returns ``(o [C*q,H,dh], lse [C*q,H] or None)``.
@@ -367,6 +389,7 @@ def rocs_dca_forward_expand(*args, expand_chunk=1024, **kw):
     return rocs_dca_forward(*args, expand_chunk=expand_chunk, **kw)
 
 
+@_on_tensor_device
 def rocs_dca_block_forward(s_seq, w_kv, q_c, q_r, cand_off, seq_off, q_tokens, q_req_tokens, scale, o_c=None,
                            o_r=None, lse=True, workspace=None, stream=None):
     """DCA block (both query groups of Eq. 13): K/V projected once per request with the stacked
@@ -402,6 +425,7 @@ def rocs_dca_block_forward(s_seq, w_kv, q_c, q_r, cand_off, seq_off, q_tokens, q
     return o_c, lse_c, o_r, lse_r
 
 
+@_on_tensor_device
 def rocs_proj_forward(inp, w, out=None, workspace=None, stream=None):
     """``out[M, N] = inp[M, K] . w[N, K]^T`` (bf16)."""
     lib = load_library()
@@ -420,6 +444,7 @@ def rocs_proj_forward(inp, w, out=None, workspace=None, stream=None):
     return out
 
 
+@_on_tensor_device
 def rocs_read_status(workspace, stream=None):
     """Synchronise the stream and return ``(device_code, detail)`` of a workspace."""
     lib = load_library()
@@ -450,6 +475,7 @@ def rocs_align_cols(cols: int, elem_bytes: int) -> int:
     return int(load_library().rocs_align_cols(int(cols), int(elem_bytes)))
 
 
+@_on_tensor_device
 def rocs_pad_cols(src, ld_dst, dst=None, stream=None):
     """Copy the rows of ``src`` (last axis contiguous) into rows of ``ld_dst`` elements, zero-filling the
     tail (section 4.2.4).  With ``ld_dst`` smaller than the source's last axis the rows are cut instead."""
@@ -465,6 +491,7 @@ def rocs_pad_cols(src, ld_dst, dst=None, stream=None):
     return dst
 
 
+@_on_tensor_device
 def rocs_fm_forward(x_req, x_cand, cand_off, y_req=None, y_cand=None, ld_req=0, ld_cand=0, workspace=None,
                     stream=None):
     """IKBO masked FM (Eq. 10).  Returns ``(y_req [R, n_r, ld_req], y_cand [C, n_c, ld_cand])``: the outputs
@@ -497,6 +524,7 @@ def rocs_fm_forward(x_req, x_cand, cand_off, y_req=None, y_cand=None, ld_req=0, 
     return y_req, y_cand
 
 
+@_on_tensor_device
 def rocs_chain_prepare_weights(w_q, w_rr, w_cr, w_cc, d, stream=None):
     """Once per model: ``(w_fold [n_out, n_c*d], w_rs [o_r + o_c, n_r])`` for :func:`rocs_chain_split_forward`."""
     lib = load_library()
@@ -513,6 +541,7 @@ def rocs_chain_prepare_weights(w_q, w_rr, w_cr, w_cc, d, stream=None):
     return w_fold, w_rs
 
 
+@_on_tensor_device
 def rocs_chain_split_forward(x_req, x_cand, w_rs, w_q, w_fold, cand_off, o_r, y_req=None, q=None, workspace=None,
                              stream=None):
     """Split chain queries: ``(y_req [R, o_r + o_c, d] = [Y^R; Z], q [C, n_out])``; see the header."""
@@ -565,6 +594,7 @@ def _host_tensor(t, what):
         raise RocsError(1, f"{what} must be a contiguous pinned host tensor")
 
 
+@_on_tensor_device
 def rocs_lcb_forward_host(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req=None, y_cand=None, chunks=8,
                           staging=None, stream=None):
     """IKBO-LCB on a host-resident batch: pinned host ``x_req``/``x_cand`` in, pinned host ``y_req``/``y_cand``
@@ -600,6 +630,7 @@ def rocs_lcb_forward_host(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, y_req=None,
     return y_req, y_cand
 
 
+@_on_tensor_device
 def rocs_dca_forward_host(q_t, k_t, v_t, cand_off, seq_off, q_tokens, scale, o=None, lse=True, device="cuda",
                           chunks=4, staging=None, stream=None):
     """IKBO-DCA on a host-resident batch: pinned host Q/K/V in, pinned host O (and LSE) out."""

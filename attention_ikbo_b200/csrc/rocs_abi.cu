@@ -2,6 +2,7 @@
 // validation, workspace layout, TMA tensor-map construction and kernel launches.
 // No entry point allocates or frees memory or synchronises a stream (except
 // rocs_read_status, whose job is to synchronise and read).
+#include <atomic>
 #include <cmath>
 #include <mutex>
 #include <cstring>
@@ -42,13 +43,18 @@ AuxStream* aux_stream_for_current_device() {
   return &x;
 }
 
+// SM count of the calling thread's current device, cached per device (threads that race on a first call
+// store the same value).
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) != cudaSuccess) return n;
-  static int cache[64] = {0};
-  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  static std::atomic<int> cache[64] = {};
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c) return c;
+  }
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  if (dev >= 0 && dev < 64) cache[dev] = n;
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 

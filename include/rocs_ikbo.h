@@ -280,6 +280,10 @@ typedef struct {
   int64_t kv_ld; /* row stride of K and V in elements; 0 = H*dh */
 } rocs_dca_args;
 
+/* The size depends on the current device's SM count (the units of the last partial wave are split in
+ * two along the keys when every request has the same number of K/V tiles, and each split unit needs a
+ * merge area): query it with the device current that rocs_dca_forward will run on.  Returns 0 when
+ * the arguments are invalid. */
 ROCS_API size_t rocs_dca_workspace_size(const rocs_dca_args* args);
 
 /* IKBO-DCA forward: a scheduling kernel (work-unit table, longest request first) and the
