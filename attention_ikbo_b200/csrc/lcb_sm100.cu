@@ -37,13 +37,20 @@ constexpr int kWarpsPerGroup = 4;  // one epilogue group covers the 128 TMEM lan
 // NG epilogue groups of four warps, then the TMA producer warp and the tcgen05 issuer warp.
 // NG = 1: the group drains both TMEM accumulator buffers in turn; NG = 2: group g drains buffer g
 // only, so two tiles' epilogues run at once (used by the block epilogue, whose per-row work is long).
+// NG = 2 launches a third full warpgroup (producer, issuer, two idle warps) so that setmaxnreg can
+// move registers from it to the epilogue warps, which hold a whole output row in registers:
+//   4 warps x 32 x kRegsCtl + 8 warps x 32 x kRegsEpi == 384 x kLaunchRegs,
+// and per SM sub-partition (warps w, w+4, w+8) kRegsCtl + 2 kRegsEpi == 3 kLaunchRegs.
 template <int NG>
 struct LcbRoles {
   static constexpr int kEpiWarps = kWarpsPerGroup * NG;
   static constexpr int kProducerWarp = kEpiWarps;
   static constexpr int kMmaWarp = kEpiWarps + 1;
-  static constexpr int kThreads = 32 * (kEpiWarps + 2);
+  static constexpr int kThreads = NG == 2 ? 384 : 32 * (kEpiWarps + 2);
+  static constexpr uint32_t kLaunchRegs = 168, kRegsCtl = 40, kRegsEpi = 232;
 };
+static_assert(4 * 32 * LcbRoles<2>::kRegsCtl + 8 * 32 * LcbRoles<2>::kRegsEpi ==
+                  LcbRoles<2>::kThreads * LcbRoles<2>::kLaunchRegs, "register split");
 constexpr uint32_t kSlot = 32768;  // one ring slot: a request k-block (A 16 KB + B <=16 KB) or one X^C tile
 constexpr int OC = 128;
 
@@ -149,7 +156,10 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
 
-  if (warp == kProducerWarp) {
+  if (warp >= kEpiWarps) {
+   // NG = 2: warpgroup 2 hands registers to the epilogue warpgroups, then producer / issuer / idle
+   if constexpr (NG == 2) reg_dealloc<LcbRoles<NG>::kRegsCtl>();
+   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       if (cbeg < cend) tma_prefetch_desc(&p.tm_xc);
@@ -254,8 +264,10 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
       umma_commit(drain_bar);  // wait for every MMA this thread issued before TMEM is freed
       mbar_drain(drain_bar, 0, 50000000ull);
     }
+   }
   } else {
     // ------------------------------------------------------------------ epilogue warps
+    if constexpr (NG == 2) reg_alloc<LcbRoles<NG>::kRegsEpi>();
     const int ew = warp;                 // epilogue warp index: staging buffers, residual barrier
     const int quarter = warp & 3;        // owns TMEM lanes / tile rows 32*quarter .. 32*quarter+31
     const int grp = warp >> 2;           // NG = 2: drains accumulator buffer grp only
@@ -581,11 +593,57 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
             rph ^= 1;
           }
           tc_fence_after();
-          epilogue_row(std::integral_constant<int, EPI_C>{}, tmem_base + t_lane + ab * D, true, 0.0f, res, stg,
-                       p.epi_c);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          if (p.epi_c.norm != EPI_NORM_NONE) {
+            // the whole row in registers: acc and Z read from TMEM once, the accumulator handed back to the
+            // MMA before any arithmetic, then exact row statistics, norm, activation and the bf16 store
+            float2 xr[D / 2];
+            const uint32_t acc = tmem_base + t_lane + ab * D;
+#pragma unroll
+            for (int q = 0; q < D / 16; ++q) {
+              uint32_t v[16], z[16];
+              tmem_ld16(acc + q * 16, v);
+              tmem_ld16(z_tmem + q * 16, z);
+              tmem_ld_wait();
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                xr[q * 8 + k] = __fadd2_rn(make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])),
+                                           make_float2(__uint_as_float(z[2 * k]), __uint_as_float(z[2 * k + 1])));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+            if (res) {
+#pragma unroll
+              for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+                for (int c16 = 0; c16 < 8; ++c16) {
+                  const uint4 u = ld_shared_v4(stg + c * L::kStgHalf + lane * 128 + ((c16 ^ (lane & 7)) << 4));
+                  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                  for (int j = 0; j < 4; ++j)
+                    xr[c * 32 + c16 * 4 + j] = __fadd2_rn(
+                        xr[c * 32 + c16 * 4 + j],
+                        make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u)));
+                }
+            }
+            RowStats st{0.0f, 0.0f, 0.0f};
+            stats_add_chunk(st, xr, p.epi_c.norm);
+            float mean, inv;
+            stats_finish(st, D, p.epi_c, mean, inv);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              float2(&xs)[32] = *reinterpret_cast<float2(*)[32]>(&xr[c * 32]);
+              norm_chunk_smem(xs, s_gb + c * 64, s_gb + D + c * 64, mean, inv);
+              act_chunk<EPI_C>(xs);
+              stage_chunk_f(stg, c, xs);
+            }
+          } else {
+            epilogue_row(std::integral_constant<int, EPI_C>{}, tmem_base + t_lane + ab * D, true, 0.0f, res, stg,
+                         p.epi_c);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          }
           store_tile(&p.tm_yc, stg_off, i * OC + 32 * quarter, true);
           // this group's next tile: its residual rows into the other staging buffer (whose last store,
           // two groups back, must have finished reading it)
@@ -620,6 +678,16 @@ static cudaError_t launch_t(const LcbParams& p, int grid, cudaStream_t st) {
   using L = LcbSmem<D, NC, NG>;
   auto k = rocs_lcb_sm100_kernel<D, NC, EPI_C, NG>;
   static std::atomic<uint64_t> optin_done{0};  // per instantiation, one bit per device
+  if constexpr (NG == 2) {
+    static std::atomic<int> regs_checked{0};  // a property of the binary: checked once per process
+    if (!regs_checked.load(std::memory_order_acquire)) {
+      // the setmaxnreg split is only valid for the register count it was computed for
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, k) != cudaSuccess || fa.numRegs != (int)LcbRoles<NG>::kLaunchRegs)
+        return cudaErrorInvalidConfiguration;
+      regs_checked.store(1, std::memory_order_release);
+    }
+  }
   cudaError_t e = ensure_smem_optin(optin_done, k, (int)L::alloc_bytes);
   if (e != cudaSuccess) return e;
   return launch_dependent(k, grid, LcbRoles<NG>::kThreads, L::alloc_bytes, st, p);
