@@ -20,6 +20,10 @@
 //     Candidates are split into equal contiguous ranges, one per CTA (all candidate tiles
 //     cost the same), which also keeps one request's Z resident for many tiles.
 //   * 4.2.4 alignment: rows are 16-byte multiples by contract, so every operand moves by TMA.
+//   * block epilogue (section 3.1.3, Eq. (7)-(8)): the candidate residual is accumulated by the tensor
+//     core (an identity A operand against the residual tile, loaded with X^C), and each epilogue warp
+//     reads its rows from TMEM once, hands the accumulator back and runs bias/norm/activation from
+//     registers (setmaxnreg moves registers to the epilogue warpgroups).
 //
 // Tile shapes: M = 128 output rows (o_c, or a 128-row slice of o_r), N = d, K = n_c for a
 // candidate tile (K-blocks of 64 for request tiles, K = n_r).  A = weights (K-major),
@@ -47,7 +51,7 @@ struct LcbRoles {
   static constexpr int kProducerWarp = kEpiWarps;
   static constexpr int kMmaWarp = kEpiWarps + 1;
   static constexpr int kThreads = NG == 2 ? 384 : 32 * (kEpiWarps + 2);
-  static constexpr uint32_t kLaunchRegs = 168, kRegsCtl = 40, kRegsEpi = 232;
+  static constexpr uint32_t kLaunchRegs = 168, kRegsCtl = 56, kRegsEpi = 224;
 };
 static_assert(4 * 32 * LcbRoles<2>::kRegsCtl + 8 * 32 * LcbRoles<2>::kRegsEpi ==
                   LcbRoles<2>::kThreads * LcbRoles<2>::kLaunchRegs, "register split");
@@ -57,17 +61,27 @@ constexpr int OC = 128;
 template <int D, int NC, int NG>
 struct LcbSmem {
   static constexpr int kEpiWarps = LcbRoles<NG>::kEpiWarps;
-  // NG = 2 (block epilogue): two staging buffers per warp so the next tile's residual rows load while this
-  // tile is finished; the ring gives up two stages for them
-  static constexpr int kStages = NG == 2 ? 2 : 4;
-  static constexpr int kStgPerWarp = 2;                   // staging buffers per epilogue warp
   static constexpr uint32_t kWcc = NC * OC * 2;           // W_CC resident, NC/64 boxes of [128 x 64]
   static constexpr uint32_t kXc = NC * D * 2;             // one candidate's X^C tile
+  static constexpr uint32_t kRes = OC * D * 2;            // one candidate's residual tile [o_c x d]
+  static constexpr uint32_t kEye = OC * OC * 2;           // identity [128 x 128], K-major A operand
   static constexpr uint32_t kStgHalf = 32 * 128;          // 32 rows x 64 bf16 (one TMA store box)
   static constexpr uint32_t kStgBuf = (D / 64) * kStgHalf;  // one warp's 32-row output tile
+  // Block epilogue (NG = 2): where shared memory allows, the candidate residual is added by the tensor
+  // core, Y^C += I . Res (an identity A operand against the residual tile as B, both bf16, accumulated
+  // in fp32: every product is exact), so its rows travel with X^C through the ring and the epilogue
+  // warps need one staging buffer each.  Otherwise two staging buffers per warp, so the next tile's
+  // residual rows load while this tile is finished, and the ring gives up two stages for them.
+  static constexpr bool kResMma =
+      NG == 2 && kWcc + kEye + 2 * (kXc + kRes) + 8 * kStgBuf + 2 * D * 4 + 2048 <= 232448 - 1024;
+  static constexpr int kStages = NG == 2 ? 2 : 4;
+  static constexpr int kStgPerWarp = kResMma ? 1 : 2;     // staging buffers per epilogue warp
+  // one ring slot: a request k-block (A 16 KB + B <= 16 KB) or one X^C tile (+ its residual tile)
+  static constexpr uint32_t kSlotSz = kResMma && kXc + kRes > kSlot ? kXc + kRes : kSlot;
   static constexpr uint32_t off_wcc = 0;
-  static constexpr uint32_t off_ring = kWcc;
-  static constexpr uint32_t off_stg = off_ring + kStages * kSlot;
+  static constexpr uint32_t off_eye = kWcc;
+  static constexpr uint32_t off_ring = off_eye + (kResMma ? kEye : 0);
+  static constexpr uint32_t off_stg = off_ring + kStages * kSlotSz;
   static constexpr uint32_t off_par = off_stg + kEpiWarps * kStgPerWarp * kStgBuf;
   static constexpr uint32_t kPar = NG == 2 ? 2 * D * 4 : 0;  // block epilogue: candidate gamma, beta (fp32)
   static constexpr uint32_t off_bar = off_par + kPar;
@@ -78,6 +92,7 @@ struct LcbSmem {
   static constexpr uint32_t tmem_cols = ((2 + NG) * D <= 256) ? 256 : 512;  // 2 accumulators + NG Z slots
   static_assert((2 + NG) * D <= 512, "tensor memory budget");
   static_assert(kXc <= kSlot, "X^C tile must fit one slot");
+  static_assert(kSlotSz % 1024 == 0 && off_ring % 1024 == 0, "swizzled operands need 1024-byte alignment");
   static_assert(alloc_bytes <= 232448, "shared memory budget");
 };
 
@@ -150,6 +165,23 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
         s_gb[k] = p.epi_c.gamma ? p.epi_c.gamma[k] : 1.0f;
         s_gb[D + k] = p.epi_c.beta ? p.epi_c.beta[k] : 0.0f;
       }
+    if constexpr (L::kResMma) {
+      // identity A operand in the layout a 128-byte-swizzled TMA load of [128 rows x 64] boxes gives:
+      // row m of box b at b*16 KB + m*128 bytes, its 16-byte chunk j stored at position j ^ (m & 7)
+      if (threadIdx.x < OC) {
+        const uint32_t m = threadIdx.x;
+        uint8_t* s_eye = smem + L::off_eye;
+#pragma unroll
+        for (uint32_t bx = 0; bx < OC / 64; ++bx)
+#pragma unroll
+          for (uint32_t j = 0; j < 8; ++j) {
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
+            if (bx == (m >> 6) && j == ((m & 63) >> 3)) w[(m & 7) >> 1] = (m & 1) ? 0x3F800000u : 0x00003F80u;
+            st_shared_v4(smem_u32(s_eye + bx * 16384 + m * 128 + ((j ^ (m & 7)) << 4)), w[0], w[1], w[2], w[3]);
+          }
+        fence_proxy_async_smem();
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -188,7 +220,7 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
         else { const int u = item - R; r = u / mt_r; arow = (u % mt_r) * OC; tmA = &p.tm_wrr; }
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, ctl, 102)) { ok = false; break; }
-          uint8_t* slot = s_ring + s * kSlot;
+          uint8_t* slot = s_ring + s * L::kSlotSz;
           mbar_arrive_expect_tx(&full[s], 16384 + 64 * D * 2);
           tma_load_2d(slot, tmA, &full[s], kb * 64, arow);
           for (int cc = 0; cc < D / 64; ++cc)
@@ -199,13 +231,17 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
       }
       for (int i = cbeg; ok && i < cend; ++i) {  // candidate phase
         if (!mbar_wait(&empty[s], ph ^ 1, ctl, 103)) { ok = false; break; }
-        uint8_t* slot = s_ring + s * kSlot;
-        mbar_arrive_expect_tx(&full[s], L::kXc);
+        uint8_t* slot = s_ring + s * L::kSlotSz;
+        const bool res_mma = L::kResMma && p.epi_c.has_residual;
+        mbar_arrive_expect_tx(&full[s], L::kXc + (res_mma ? L::kRes : 0u));
         for (int cc = 0; cc < D / 64; ++cc) {
           // LCB block: X^C is read once; evict-first keeps the residual rows prefetched for the epilogue in L2
           if constexpr (EPI) tma_load_2d_hint(slot + cc * (NC * 128), &p.tm_xc, &full[s], cc * 64, i * NC, l2_evict_first());
           else tma_load_2d(slot + cc * (NC * 128), &p.tm_xc, &full[s], cc * 64, i * NC);
         }
+        if (res_mma)  // the residual tile [o_c rows x d] as the B operand of Y^C += I . Res (read once)
+          for (int cc = 0; cc < D / 64; ++cc)
+            tma_load_2d_hint(slot + L::kXc + cc * (OC * 128), &p.tm_res_cb, &full[s], cc * 64, i * OC, l2_evict_first());
         ++n_issued;
         if (++s == L::kStages) { s = 0; ph ^= 1; }
       }
@@ -233,7 +269,7 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
         for (int kb = 0; kb < kblocks && ok; ++kb) {
           if (!mbar_wait(&full[s], ph, ctl, 203)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(s_ring + s * kSlot);
+          const uint32_t a0 = smem_u32(s_ring + s * L::kSlotSz);
           const uint64_t ad = sdesc_sw128(a0, 16, 1024), bd = sdesc_sw128(a0 + 16384, 8192, 1024);
 #pragma unroll
           for (int kin = 0; kin < 4; ++kin)
@@ -247,15 +283,23 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
       }
       if (ok && cbeg < cend && !mbar_wait(wcc_bar, 0, ctl, 204)) ok = false;
       const uint64_t wccd = sdesc_sw128(smem_u32(s_wcc), 16, 1024);
+      const uint64_t eyed = sdesc_sw128(smem_u32(smem + L::off_eye), 16, 1024);
+      const bool res_mma = L::kResMma && p.epi_c.has_residual;
       for (int i = cbeg; ok && i < cend; ++i) {  // candidate tiles
         if (!mbar_wait(&acc_empty[ab], aph ^ 1, ctl, 205)) { ok = false; break; }
         if (!mbar_wait(&full[s], ph, ctl, 206)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * D;
-        const uint64_t bd = sdesc_sw128(smem_u32(s_ring + s * kSlot), NC * 128, 1024);
+        const uint64_t bd = sdesc_sw128(smem_u32(s_ring + s * L::kSlotSz), NC * 128, 1024);
 #pragma unroll
         for (int ks = 0; ks < NC / 16; ++ks)
           umma_ss(d_tmem, sdesc_add(wccd, (ks >> 2) * 16384 + (ks & 3) * 32), sdesc_add(bd, ks * 2048), idesc, ks != 0);
+        if (res_mma) {  // Y^C += I . Res: K runs over the residual tile's o_c rows
+          const uint64_t rd = sdesc_sw128(smem_u32(s_ring + s * L::kSlotSz + L::kXc), OC * 128, 1024);
+#pragma unroll
+          for (int ks = 0; ks < OC / 16; ++ks)
+            umma_ss(d_tmem, sdesc_add(eyed, (ks >> 2) * 16384 + (ks & 3) * 32), sdesc_add(rd, ks * 2048), idesc, 1u);
+        }
         umma_commit(&empty[s]);
         umma_commit(&acc_full[ab]);
         if (++s == L::kStages) { s = 0; ph ^= 1; }
@@ -570,10 +614,11 @@ __global__ void __launch_bounds__(LcbRoles<NG>::kThreads, 1) rocs_lcb_sm100_kern
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);
           store_tile(&p.tm_yc, stg_off, i * OC + 32 * quarter);
-        } else {  // candidate group's epilogue: residual loaded one tile ahead into the other staging buffer
+        } else {  // candidate group's epilogue (a residual either in the accumulator already, see kResMma,
+                  // or loaded one tile ahead into the warp's other staging buffer)
           const uint32_t stg_off = acquire_stage();
           const uint32_t stg = smem_u32(s_stg + stg_off);
-          const bool res = p.epi_c.has_residual != 0;
+          const bool res = !L::kResMma && p.epi_c.has_residual != 0;
           if (res) {
             if (res_next != i) load_residual(&p.tm_res_c, stg_off, i * OC + 32 * quarter);
             // this group's tile after next: start its residual rows towards L2 now

@@ -23,6 +23,7 @@ struct LcbParams {
   // LCB block epilogue (used by the epilogue instantiation only)
   CUtensorMap tm_res_r;     // residual of Y^R viewed as [R*o_r, d], box {64, 32} (loads)
   CUtensorMap tm_res_c;     // residual of Y^C viewed as [C*o_c, d], box {64, 32} (loads)
+  CUtensorMap tm_res_cb;    // the same, box {64, 128}: one candidate's whole residual tile (B operand loads)
   EpiGroup epi_r, epi_c;
 };
 // Zeroes a[0:na] and b[0:nb] (the workspace header and the request ready flags) and lets the LCB kernel that

@@ -241,10 +241,13 @@ int lcb_run(const rocs_lcb_args* a, int64_t C, WsHeader* hdr, uint8_t* w, cudaSt
     // residual maps: the same boxes as the output stores (unused maps get any valid descriptor)
     p.tm_res_r = p.tm_yr;
     p.tm_res_c = p.tm_yr;
+    p.tm_res_cb = p.tm_yr;
     if (p.epi_r.has_residual)
       ok &= tmap_bf16(&p.tm_res_r, opts.epi_r->residual, d, (uint64_t)a->R * a->o_r, rb, 64, 32);
-    if (p.epi_c.has_residual && C > 0)
+    if (p.epi_c.has_residual && C > 0) {
       ok &= tmap_bf16(&p.tm_res_c, opts.epi_c->residual, d, (uint64_t)C * a->o_c, rb, 64, 32);
+      ok &= tmap_bf16(&p.tm_res_cb, opts.epi_c->residual, d, (uint64_t)C * a->o_c, rb, 64, 128);
+    }
   }
   if (!ok) return ROCS_ERR_CUDA;
   p.cand_off = a->cand_off_dev;

@@ -59,6 +59,7 @@ CASES = [  # (counts, n_r, n_c, d, o_r, norm, act, residual)
     ([9, 33, 0, 2], 64, 64, 64, 256, "layernorm", "relu", False),
     ([150, 151], 128, 128, 64, 128, "none", "gelu", True),
     ([0, 0, 4], 64, 64, 128, 128, "rmsnorm", "none", False),
+    ([5, 70, 0, 3], 128, 64, 64, 128, "layernorm", "silu", True),
 ]
 
 
