@@ -44,6 +44,7 @@ from ._binding import (  # noqa: F401
     rocs_dca_forward_host,
     rocs_fm_forward,
     rocs_lcb_block_forward,
+    rocs_lcb_block_forward_fault_injection,
     rocs_lcb_forward,
     rocs_lcb_forward_expand,
     rocs_lcb_forward_fault_injection,

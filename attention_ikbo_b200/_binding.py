@@ -105,6 +105,8 @@ def load_library():
                            ("rocs_lcb_forward_noalloc", [P(LcbArgs), _vp]),
                            ("rocs_lcb_block_forward", [P(LcbArgs), P(LcbEpilogue), P(LcbEpilogue), _vp]),
                            ("rocs_lcb_forward_fault_injection", [P(LcbArgs), _vp, _i64, _i64]),
+                           ("rocs_lcb_block_forward_fault_injection",
+                            [P(LcbArgs), P(LcbEpilogue), P(LcbEpilogue), _vp, _i64, _i64]),
                            ("rocs_dca_forward", [P(DcaArgs), _vp]), ("rocs_proj_forward", [P(ProjArgs), _vp]),
                            ("rocs_dca_forward_expand", [P(DcaArgs), _i64, _vp]),
                            ("rocs_dca_block_forward", [P(DcaBlockArgs), _vp]),
@@ -329,6 +331,24 @@ def rocs_lcb_block_forward(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, epi_req=No
            "rocs_lcb_block_forward")
     rocs_lcb_block_forward.last_workspace = ws
     return y_req, y_cand
+
+
+@_on_tensor_device
+def rocs_lcb_block_forward_fault_injection(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, epi_req, epi_cand,
+                                           skip_release_request, wait_limit_ns, stream=None):
+    """Test hook: LCB block whose request ``skip_release_request`` never signals its Z; the kernel must
+    end with ROCS_ERR_TIMEOUT after ``wait_limit_ns``.  Returns the workspace (read it with rocs_read_status)."""
+    lib = load_library()
+    a, keep, y_req, y_cand = _lcb_args(x_req, x_cand, w_rr, w_cr, w_cc, cand_off, None, None)
+    hold = []
+    er = _epilogue(epi_req, tuple(y_req.shape), x_req.device, hold)
+    ec = _epilogue(epi_cand, tuple(y_cand.shape), x_req.device, hold)
+    ws = _workspace(lib.rocs_lcb_workspace_size(ctypes.byref(a)), x_req.device, None)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check(lib.rocs_lcb_block_forward_fault_injection(
+        ctypes.byref(a), None if er is None else ctypes.byref(er), None if ec is None else ctypes.byref(ec),
+        _stream(stream), int(skip_release_request), int(wait_limit_ns)), "rocs_lcb_block_forward_fault_injection")
+    return ws
 
 
 def rocs_lcb_forward_expand(*args, **kw):

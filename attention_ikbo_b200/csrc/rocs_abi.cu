@@ -464,6 +464,31 @@ int rocs_lcb_forward_fault_injection(const rocs_lcb_args* a, rocs_stream_t strea
   return rc;
 }
 
+int rocs_lcb_block_forward_fault_injection(const rocs_lcb_args* a, const rocs_lcb_epilogue* epi_req,
+                                           const rocs_lcb_epilogue* epi_cand, rocs_stream_t stream,
+                                           int64_t skip_release_request, int64_t wait_limit_ns) {
+  int64_t C = 0;
+  int rc = lcb_validate(a, &C);
+  if (rc) return rc;
+  if (a->dtype != ROCS_BF16) return ROCS_ERR_UNSUPPORTED;
+  if ((rc = epi_validate(epi_req)) || (rc = epi_validate(epi_cand))) return rc;
+  if (skip_release_request < -1 || skip_release_request >= a->R) return ROCS_ERR_INVALID_ARG;
+  if (wait_limit_ns < 1000000 || wait_limit_ns > 10000000000ll) return ROCS_ERR_INVALID_ARG;
+  if (!a->workspace || a->workspace_bytes < lcb_bytes(a) || (reinterpret_cast<uintptr_t>(a->workspace) & 255))
+    return ROCS_ERR_WORKSPACE;
+  LcbOpts o;
+  o.block = true;
+  o.epi_r = epi_req;
+  o.epi_c = epi_cand;
+  o.wait_ns = wait_limit_ns;
+  o.skip_release = (int)skip_release_request;
+  int launches = 0;
+  WsHeader* hdr = static_cast<WsHeader*>(a->workspace);
+  rc = lcb_run(a, C, hdr, reinterpret_cast<uint8_t*>(hdr + 1), reinterpret_cast<cudaStream_t>(stream), &launches, o);
+  if (rc == ROCS_OK) g_last_launches = launches;
+  return rc;
+}
+
 int rocs_lcb_block_forward(const rocs_lcb_args* a, const rocs_lcb_epilogue* epi_req,
                            const rocs_lcb_epilogue* epi_cand, rocs_stream_t stream) {
   int64_t C = 0;

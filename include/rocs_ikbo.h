@@ -201,6 +201,16 @@ typedef struct {
 ROCS_API int rocs_lcb_block_forward(const rocs_lcb_args* args, const rocs_lcb_epilogue* epi_req,
                                     const rocs_lcb_epilogue* epi_cand, rocs_stream_t stream);
 
+/* Fault-injection hook for the LCB block kernel (not for production use; the paper has no
+ * counterpart): rocs_lcb_block_forward whose request tile computing Z for request
+ * `skip_release_request` (-1: none) never releases its ready flag, with every device wait limited
+ * to `wait_limit_ns` (1e6 .. 1e10).  Same contract as rocs_lcb_forward_fault_injection: the
+ * kernel ends with ROCS_ERR_TIMEOUT in the workspace status word, no trap, no hang, and the
+ * context stays usable; outputs of the affected request are undefined. */
+ROCS_API int rocs_lcb_block_forward_fault_injection(const rocs_lcb_args* args, const rocs_lcb_epilogue* epi_req,
+                                                    const rocs_lcb_epilogue* epi_cand, rocs_stream_t stream,
+                                                    int64_t skip_release_request, int64_t wait_limit_ns);
+
 /* ------------------------------------------------------------------------------------
  * IKBO masked factorization machine  (section 3.1.4 Eq. (9)-(10); section 4.1; section 4.2.4)
  *

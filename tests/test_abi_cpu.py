@@ -138,6 +138,13 @@ def test_lcb_block_host_validation(lib):
     assert lib.rocs_lcb_block_forward(P(bad), None, None, None) == 2
     small, keep4 = _lcb_args(m, [0, 3, 6], ws_bytes=100)
     assert lib.rocs_lcb_block_forward(P(small), None, None, None) == 6
+    # the block kernel's fault-injection hook validates like both of its parents
+    fi = lib.rocs_lcb_block_forward_fault_injection
+    assert fi(P(a), None, None, None, 5, 10_000_000) == 1  # no request 5
+    assert fi(P(a), None, None, None, 0, 10) == 1  # limit below 1 ms
+    assert fi(P(a), P(E(norm=3)), None, None, 0, 10_000_000) == 1  # unknown norm
+    assert fi(P(f32), None, None, None, 0, 10_000_000) == 3
+    assert fi(P(small), None, None, None, 0, 10_000_000) == 6
 
 
 def test_fm_host_validation(lib):
