@@ -74,8 +74,11 @@ struct LcbSmem {
   // residual rows load while this tile is finished, and the ring gives up two stages for them.
   static constexpr bool kResMma =
       NG == 2 && kWcc + kEye + 2 * (kXc + kRes) + 8 * kStgBuf + 2 * D * 4 + 2048 <= 232448 - 1024;
-  static constexpr int kStages = NG == 2 ? 2 : 4;
-  static constexpr int kStgPerWarp = kResMma ? 1 : 2;     // staging buffers per epilogue warp
+  // Plain LCB (NG = 1): the output stream is twice the input stream, so shared memory goes to output
+  // staging first (more TMA stores in flight per warp), then to the X^C ring: 3 stages and 3 staging
+  // buffers per warp at n_c = 64 (a 16 KB X^C tile per 32 KB slot), 2 and 4 at n_c = 128.
+  static constexpr int kStages = NG == 2 ? 2 : (NC == 64 ? 3 : 2);
+  static constexpr int kStgPerWarp = kResMma ? 1 : (NG == 1 ? (NC == 64 ? 3 : 4) : 2);  // per epilogue warp
   // one ring slot: a request k-block (A 16 KB + B <= 16 KB) or one X^C tile (+ its residual tile)
   static constexpr uint32_t kSlotSz = kResMma && kXc + kRes > kSlot ? kXc + kRes : kSlot;
   static constexpr uint32_t off_wcc = 0;
