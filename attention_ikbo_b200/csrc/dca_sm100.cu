@@ -709,15 +709,21 @@ __global__ void __launch_bounds__(kThreads, 1) rocs_dca_sm100_kernel(const __gri
 // length descending (ties by index) so the longest units are claimed first.  The last n_split units
 // in that order (the shortest) become two entries each, the halves of their K/V tiles, so that the
 // final partial wave of the persistent grid is made of half-length work.
-// Scratch (workspace): len[R], sorted[R], start[R+1] (first unit of each sorted position, then the total).
+// Per-request arrays len[R], sorted[R], start[R+1] (first unit of each sorted position, then the total): in
+// shared memory for R <= 2048, else in the workspace scratch.
 // ------------------------------------------------------------------------------------
 __global__ void rocs_dca_schedule_kernel(const DcaSchedParams p) {
   // the attention kernel may start its prologue now; it waits for this grid before claiming units
   asm volatile("griddepcontrol.launch_dependents;");
-  int* len = p.scratch;
-  int* sorted = len + p.R;
-  int* start = sorted + p.R;
+  // per-request arrays in shared memory when they fit (every phase below reads them back, the last one by
+  // binary search), else in the workspace scratch
+  constexpr int kSmemR = 2048;
   __shared__ int s_part[1024];
+  __shared__ int s_len[kSmemR], s_sorted[kSmemR], s_start[kSmemR + 1];
+  const bool in_smem = p.R <= kSmemR;
+  int* len = in_smem ? s_len : p.scratch;
+  int* sorted = in_smem ? s_sorted : p.scratch + p.R;
+  int* start = in_smem ? s_start : p.scratch + 2 * p.R;
   const int R = p.R, T = blockDim.x, t = threadIdx.x;
   for (int r = t; r < R; r += T) len[r] = p.seq_off[r + 1] - p.seq_off[r];
   __syncthreads();
