@@ -92,6 +92,51 @@ def test_dca_host_validation(lib):
     assert lib.rocs_dca_forward(ctypes.byref(a), None) == 3
 
 
+def test_dca_workspace_counts_split_and_paired_units(lib):
+    """Host logic of the DCA schedule, pinned through the workspace size (no GPU: the SM count falls back to
+    148).  Units = H * ceil(q N_r / 256); when every request has the same number (>= 2) of K/V tiles the last
+    (units mod 148) units are split in two (one more table entry each, plus 8 counters and a merge area of
+    2 halves x 2 tiles x 4 warps x 32 rows x (dh + 2) fp32); at dh = 64 a request's last chunk of <= 128 rows
+    is one unit per head pair."""
+    import attention_ikbo_b200 as m
+
+    fake = 0x20000
+    a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+
+    def size(counts, lengths, H, dh, q=1):
+        co = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        so = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+        a = m._binding.DcaArgs(R=len(counts), q=q, H=H, dh=dh, scale=0.1, cand_off_dev=fake,
+                               cand_off_host=co.ctypes.data, seq_off_dev=fake, seq_off_host=so.ctypes.data,
+                               q_ptr=fake, k_ptr=fake, v_ptr=fake, o_ptr=fake, lse_ptr=None, workspace=None,
+                               workspace_bytes=0)
+        return lib.rocs_dca_workspace_size(ctypes.byref(a))
+
+    def expect(R, n_units, n_split, dh):
+        units = a256((3 * R + 1) * 4)
+        body = units + (n_units + n_split) * 16
+        if n_split:
+            split_buf = a256(a256(body) + n_split * 8 * 4)
+            body = split_buf + n_split * 2 * 2 * 4 * 32 * (dh + 2) * 4
+        return 256 + body
+
+    # 10 requests x 8 heads x 2 chunks = 160 units, all with 3 K/V tiles: 160 mod 148 = 12 split
+    assert size([512] * 10, [300] * 10, 8, 128) == expect(10, 160, 12, 128)
+    # one request with a different key count: no split
+    assert size([512] * 10, [300] * 9 + [420], 8, 128) == expect(10, 160, 0, 128)
+    # a single K/V tile per request cannot be split
+    assert size([512] * 10, [100] * 10, 8, 128) == expect(10, 160, 0, 128)
+    # a multiple of 148 units leaves no partial wave
+    assert size([256] * 37, [300] * 37, 4, 128) == expect(37, 148, 0, 128)
+    # dh = 64: 100 rows (one chunk <= 128 rows) for 16 heads -> 8 head-pair units; dh = 128: 16 units
+    assert size([100], [1000], 16, 64) == expect(1, 8, 0, 64)
+    assert size([100], [1000], 16, 128) == expect(1, 16, 0, 128)
+    # dh = 64, 300 rows: two chunks, the second of 44 rows paired -> 16 + 8 units; an odd head count keeps
+    # its last head alone
+    assert size([300], [1000], 16, 64) == expect(1, 24, 0, 64)
+    assert size([300], [1000], 15, 64) == expect(1, 15 + 8, 0, 64)
+
+
 def test_proj_host_validation(lib):
     import attention_ikbo_b200 as m
 
